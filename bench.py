@@ -1,0 +1,449 @@
+"""Benchmark of the recurrent gated-delta-rule decode step on B200.
+
+One step = one call of the fused-gate decode (every step of the op: gather the
+state slot, gate prologue, decay, memory read, delta update, output, padding,
+scatter) over one batch of seeded synthetic inputs of the large-batch workload
+(B=512 items, 64 heads, T=1, 64x512 bfloat16 state per head, 2 GiB pool).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdr|reference]
+
+Prints one JSON line (rank 0). Multi-GPU: one process per GPU under torchrun;
+each rank decodes its own independent batch and pool (weak scaling, no
+collective on the data path); the timed region is bracketed by barriers and
+the max over ranks is reported.
+
+``--impl reference`` times the CPU oracle (fp64 NumPy) on this machine's host
+cores on a bounded sample of the same workload; it is a deliberately slow
+baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gated_delta_rule_recurrent_b200 import metrics, workloads  # noqa: E402
+
+METRIC = "decode tokens/s and achieved HBM GB/s vs ~8 TB/s peak for gated-delta step"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+DEFAULT_WORKLOAD = 4
+KERNEL_SOURCE_FILES = ("gated_delta_rule_recurrent_b200/csrc/gdr_decode.cuh",
+                       "gated_delta_rule_recurrent_b200/csrc/gdr_api.cu")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gated_B512_H64_64x512_dram.txt")
+
+
+# --------------------------------------------------------------------------- helpers
+
+def _dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            peaks = json.load(f)
+        return float(peaks["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCE_FILES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        rec = {}
+        with open(TRAFFIC_RECORD) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    rec[k.strip()] = v.strip()
+        if rec.get("kernel_source_sha256") != kernel_source_hash():
+            return None
+        return int(float(rec["dram_bytes_per_launch"]))
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every ``period_ms``."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, period_ms: int = 50):
+        self.samples = []  # (host time, sm_mhz, max_mhz, power, reasons set)
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            cmd = ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}",
+                   "--format=csv,noheader,nounits", f"-lms={period_ms}"]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, smax, power = float(parts[0]), float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                     "sw_power_cap"]
+            reasons = {n for n, v in zip(names, parts[4:8]) if v.lower().startswith("active")}
+            self.samples.append((time.time(), sm, smax, power, reasons))
+
+    def wait_first(self, timeout=10.0):
+        t0 = time.time()
+        while self.proc is not None and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.02)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "window": "unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if not inside:  # timed region shorter than the sampling period
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            window = "nearest to timed region"
+        reasons = sorted(set().union(*[s[4] for s in inside]))
+        return {"sm_mhz": float(np.median([s[1] for s in inside])),
+                "sm_max_mhz": max(s[2] for s in inside),
+                "power_w_max": max(s[3] for s in inside),
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+def oracle_tokens_per_s(x, gated, items_per_call, budget_s, items_order=None):
+    """Time the fp64 oracle on consecutive chunks of batch items until ``budget_s``."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle.gdr_oracle import (recurrent_gated_delta_rule,
+                                   recurrent_gated_delta_rule_gated)
+
+    B = x["query"].shape[0]
+    order = np.arange(B) if items_order is None else items_order
+    asl = x["actual_seq_lengths"].to(torch.int64).numpy()
+    idx = x["ssm_state_indices"].to(torch.int64).numpy()
+    T = x["query"].shape[2]
+
+    def f64(t):
+        return t.to(torch.float64).numpy()
+
+    tokens = 0
+    items_done = 0
+    elapsed = 0.0
+    pos = 0
+    with threadpool_limits(limits=1):
+        while elapsed < budget_s:
+            sel = order[pos:pos + items_per_call]
+            if sel.size == 0:
+                pos = 0
+                continue
+            pos += items_per_call
+            st = torch.from_numpy(idx[sel])
+            pool = f64(x["state_pool"][st])  # gathered slots (inputs, not timed)
+            args = {k: f64(x[k][torch.from_numpy(sel)]) for k in
+                    ("query", "key", "value", "gk", "a", "b", "beta", "g")}
+            local_idx = np.arange(sel.size)
+            t0 = time.perf_counter()
+            if gated:
+                recurrent_gated_delta_rule_gated(
+                    args["query"], args["key"], args["value"], args["a"], args["b"],
+                    f64(x["dt_bias"]), f64(x["decay_scale"]), pool, asl[sel], local_idx,
+                    args["gk"], asl[sel], x["scale_value"])
+            else:
+                recurrent_gated_delta_rule(
+                    args["query"], args["key"], args["value"], args["beta"], pool, asl[sel],
+                    local_idx, args["g"], args["gk"], asl[sel], x["scale_value"])
+            elapsed += time.perf_counter() - t0
+            tokens += int(np.clip(asl[sel], 0, T).sum())
+            items_done += sel.size
+    return tokens / elapsed, tokens, items_done, elapsed
+
+
+# --------------------------------------------------------------------------- CUDA arm
+
+def run_gdr(args):
+    import torch.distributed as dist
+
+    world, rank, local = _dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    import gated_delta_rule_recurrent_b200 as gdr
+    from gated_delta_rule_recurrent_b200 import binding
+
+    binding.lib()  # fail loudly now if the library is missing
+    w = workloads.workload(args.workload)
+    gated = w.gated
+    # Each rank decodes its own batch: independent sequences and pool slots.
+    x = workloads.make_inputs(w, seed=w.seed + 7919 * rank)
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    out = torch.empty(w.B, w.H_v, w.T, w.D_v, dtype=torch.bfloat16, device=dev)
+    lengths = x["actual_seq_lengths"].tolist()
+    n_tokens = int(sum(min(max(L, 0), w.T) for L in lengths))
+    step_bytes = metrics.algorithmic_bytes(w.B, w.H_qk, w.H_v, w.T, w.D_k, w.D_v, lengths,
+                                           gated)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(o=out):
+        if gated:
+            gdr.decode_gated(xd["query"], xd["key"], xd["value"], xd["a"], xd["b"],
+                             xd["dt_bias"], xd["decay_scale"], xd["state_pool"],
+                             xd["actual_seq_lengths"], xd["ssm_state_indices"], xd["gk"],
+                             xd["num_accepted_tokens"], xd["scale_value"], out=o)
+        else:
+            gdr.decode(xd["query"], xd["key"], xd["value"], xd["beta"], xd["state_pool"],
+                       xd["actual_seq_lengths"], xd["ssm_state_indices"], xd["g"], xd["gk"],
+                       xd["num_accepted_tokens"], xd["scale_value"], out=o)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    sampler = ClockSampler(local)
+    sampler.wait_first()
+
+    # ---- kernel-resident timing: inputs already in HBM
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    host_t0 = time.time()
+    region0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    region1.record(stream)
+    torch.cuda.synchronize(dev)
+    host_t1 = time.time()
+    barrier()
+    launches = K  # one kernel per step (the decode kernel)
+    region_ms = max_over_ranks(region0.elapsed_time(region1))
+    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    kernel_ms = max_over_ranks(kernel_ms)
+    clocks = sampler.summary(host_t0, host_t1)
+
+    # ---- end to end through the public API: pinned host inputs copied in and
+    # the output copied back every step, inside the timed region. The state
+    # pool stays resident on the device, as it does in serving.
+    e2e = None
+    if not args.no_e2e:
+        per_step = ["query", "key", "value", "gk", "actual_seq_lengths", "ssm_state_indices",
+                    "num_accepted_tokens"] + (["a", "b"] if gated else ["beta", "g"])
+        host = {k: x[k].pin_memory() for k in per_step}
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in per_step)
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for k in per_step:
+                xd[k].copy_(host[k], non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * n_tokens * K / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms / K}
+    sampler.stop()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, toks, items, secs = oracle_tokens_per_s(x, gated, items_per_call=8,
+                                                     budget_s=args.cpu_seconds)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{items} of {w.B} batch items ({toks} tokens) of the same "
+                         f"workload, fp64 NumPy, 1 thread, {secs:.1f} s of oracle time"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_hbm_peak()
+    achieved = step_bytes / (kernel_ms / 1e3) / 1e9
+    value = world * n_tokens * K / (region_ms / 1e3)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": region_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "H_qk": w.H_qk, "H_v": w.H_v, "T": w.T,
+            "D_k": w.D_k, "D_v": w.D_v, "pool": w.pool,
+            "gate": "fused" if gated else "none",
+            "storage": "bf16 state/q/k/v/out, fp32 g/gk",
+            "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB per step vs "
+                  f"{L2_BYTES / 2**20:.0f} MiB L2, no flush",
+            "parallelism": f"{world} independent rank(s), no collective",
+        },
+        "achieved_hbm_gbs": achieved,
+        "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth",
+            "kernel": "gdr::decode_kernel", "kernel_ms": kernel_ms,
+            "bytes_per_launch": step_bytes, "traffic": recorded_traffic(),
+        },
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- oracle arm
+
+def run_reference(args):
+    world, rank, _ = _dist_env()
+    if rank != 0:
+        return  # rank 0 alone times the CPU oracle
+    w = workloads.workload(args.workload)
+    x = workloads.make_inputs(w)
+    n_steps = args.warmup + args.steps
+    budget_total = args.reference_seconds
+    per_step_budget = budget_total / max(1, n_steps)
+    # calibrate: items per step so that every step is a bounded sample
+    tps, _, _, _ = oracle_tokens_per_s(x, w.gated, items_per_call=1, budget_s=0.5)
+    items_per_step = max(1, int(per_step_budget * tps / max(1, w.T)))
+    items_per_step = min(items_per_step, w.B)
+    order = np.arange(w.B)
+    tokens = 0
+    secs = 0.0
+    for i in range(n_steps):
+        sel = np.roll(order, -i * items_per_step)[:items_per_step]
+        _, toks, _, el = oracle_tokens_per_s(x, w.gated, items_per_call=items_per_step,
+                                             budget_s=1e-9, items_order=sel)
+        if i >= args.warmup:
+            tokens += toks
+            secs += el
+    value = tokens / secs
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H_qk": w.H_qk, "H_v": w.H_v, "T": w.T,
+                   "D_k": w.D_k, "D_v": w.D_v, "pool": w.pool,
+                   "gate": "fused" if w.gated else "none",
+                   "sample_items_per_step": items_per_step},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{items_per_step} of {w.B} batch items per step, "
+                                   f"fp64 NumPy oracle, 1 thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("gdr", "reference"), default="gdr")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    type=lambda s: int(s) if s.isdigit() else s)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "gdr":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gdr(args)
+
+
+if __name__ == "__main__":
+    main()

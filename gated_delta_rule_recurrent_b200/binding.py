@@ -1,0 +1,182 @@
+"""ctypes binding of libgdr: torch tensors in, C-ABI calls out.
+
+Only argument marshalling happens here: shape/dtype/device checks (raising
+RuntimeError as the op's page specifies in section 异常 of
+"lite_boost.ops.recurrent_gated_delta_rule"), the sizes struct, raw device
+pointers and the current CUDA stream. Every step of the computation runs in
+the library's kernels. Loading fails loudly when libgdr.so is missing; there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["decode", "decode_gated", "GdrError", "lib", "library_path", "STATUS_NAMES", "Dims"]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+
+STATUS_NAMES = {0: "GDR_OK", 1: "GDR_ERR_NULL", 2: "GDR_ERR_DIMS", 3: "GDR_ERR_ALIGN",
+                4: "GDR_ERR_UNSUPPORTED", 5: "GDR_ERR_CUDA"}
+
+
+class GdrError(RuntimeError):
+    """A libgdr entry point returned a nonzero status."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32)
+                for n in ("B", "T", "H_qk", "H_v", "D_k", "D_v", "pool_size")]
+
+
+_P = ctypes.c_void_p
+_DECODE_ARGTYPES = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                    ctypes.c_float, _P, _P]
+_GATED_ARGTYPES = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                   ctypes.c_float, _P, _P]
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.environ.get("GDR_LIBRARY", os.path.join(_PKG_DIR, "libgdr.so"))
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdr.so (loaded once; raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"libgdr.so not found at {path}; build it with "
+                "`python -m gated_delta_rule_recurrent_b200.build`")
+        L = ctypes.CDLL(path)
+        L.gdr_decode.argtypes = _DECODE_ARGTYPES
+        L.gdr_decode.restype = ctypes.c_int
+        L.gdr_gate_fused.argtypes = _GATED_ARGTYPES
+        L.gdr_gate_fused.restype = ctypes.c_int
+        L.gdr_status_string.argtypes = [ctypes.c_int]
+        L.gdr_status_string.restype = ctypes.c_char_p
+        L.gdr_last_error.argtypes = []
+        L.gdr_last_error.restype = ctypes.c_char_p
+        L.gdr_abi_version.argtypes = []
+        L.gdr_abi_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise GdrError(rc, lib().gdr_last_error().decode())
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape, device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise RuntimeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise RuntimeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise RuntimeError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise RuntimeError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise RuntimeError(f"{name} must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _common(query, key, value, state_pool, actual_seq_lengths, ssm_state_indices, gk,
+            num_accepted_tokens, out):
+    if not isinstance(query, torch.Tensor) or query.dim() != 4:
+        raise RuntimeError("query must be a 4-D tensor [B, H_qk, T, D_k]")
+    device = query.device
+    if device.type != "cuda":
+        raise RuntimeError("all tensors must be on a CUDA device")
+    B, H_qk, T, D_k = query.shape
+    if not isinstance(value, torch.Tensor) or value.dim() != 4:
+        raise RuntimeError("value must be a 4-D tensor [B, H_v, T, D_v]")
+    H_v, D_v = value.shape[1], value.shape[3]
+    if not isinstance(state_pool, torch.Tensor) or state_pool.dim() != 4:
+        raise RuntimeError("state_pool must be a 4-D tensor [pool, H_v, D_k, D_v]")
+    P = state_pool.shape[0]
+    bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    _need(query, "query", bf16, (B, H_qk, T, D_k), device)
+    _need(key, "key", bf16, (B, H_qk, T, D_k), device)
+    _need(value, "value", bf16, (B, H_v, T, D_v), device)
+    _need(state_pool, "state_pool", bf16, (P, H_v, D_k, D_v), device)
+    _need(actual_seq_lengths, "actual_seq_lengths", i32, (B,), device)
+    _need(ssm_state_indices, "ssm_state_indices", i32, (B,), device)
+    _need(gk, "gk", f32, (B, H_v, T, D_k), device)
+    if num_accepted_tokens is not None:
+        _need(num_accepted_tokens, "num_accepted_tokens", i32, (B,), device)
+    if out is None:
+        out = torch.empty((B, H_v, T, D_v), dtype=bf16, device=device)
+    else:
+        _need(out, "out", bf16, (B, H_v, T, D_v), device)
+    dims = Dims(B, T, H_qk, H_v, D_k, D_v, P)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    return device, dims, out, stream
+
+
+def decode(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, beta: torch.Tensor,
+           state_pool: torch.Tensor, actual_seq_lengths: torch.Tensor,
+           ssm_state_indices: torch.Tensor, g: torch.Tensor, gk: torch.Tensor,
+           num_accepted_tokens: Optional[torch.Tensor] = None, scale_value: float = 1.0, *,
+           out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """recurrent_gated_delta_rule decode step through ``gdr_decode``.
+
+    Argument order and defaults follow the op's page. ``state_pool`` is
+    updated in place and returned as the second result (the page's
+    ``state_out``). Queued on the current CUDA stream; no synchronisation.
+    """
+    device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
+                                        ssm_state_indices, gk, num_accepted_tokens, out)
+    B, H_v, T = dims.B, dims.H_v, dims.T
+    _need(beta, "beta", torch.bfloat16, (B, H_v, T), device)
+    _need(g, "g", torch.float32, (B, H_v, T), device)
+    with torch.cuda.device(device):
+        rc = lib().gdr_decode(ctypes.byref(dims), _ptr(query), _ptr(key), _ptr(value),
+                              _ptr(beta), _ptr(state_pool), _ptr(actual_seq_lengths),
+                              _ptr(ssm_state_indices), _ptr(g), _ptr(gk),
+                              _ptr(num_accepted_tokens), float(scale_value), _ptr(out), stream)
+    _check(rc)
+    return out, state_pool
+
+
+def decode_gated(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, a: torch.Tensor,
+                 b: torch.Tensor, dt_bias: torch.Tensor, decay_scale: torch.Tensor,
+                 state_pool: torch.Tensor, actual_seq_lengths: torch.Tensor,
+                 ssm_state_indices: torch.Tensor, gk: torch.Tensor,
+                 num_accepted_tokens: Optional[torch.Tensor] = None, scale_value: float = 1.0,
+                 *, out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Decode step with the LinearAttentionGate prologue fused, through ``gdr_gate_fused``.
+
+    ``a`` and ``b`` are [B, T, H_v] bf16; ``dt_bias`` and ``decay_scale`` are
+    [H_v] fp32. g and beta are computed inside the kernel.
+    """
+    device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
+                                        ssm_state_indices, gk, num_accepted_tokens, out)
+    B, H_v, T = dims.B, dims.H_v, dims.T
+    _need(a, "a", torch.bfloat16, (B, T, H_v), device)
+    _need(b, "b", torch.bfloat16, (B, T, H_v), device)
+    _need(dt_bias, "dt_bias", torch.float32, (H_v,), device)
+    _need(decay_scale, "decay_scale", torch.float32, (H_v,), device)
+    with torch.cuda.device(device):
+        rc = lib().gdr_gate_fused(ctypes.byref(dims), _ptr(query), _ptr(key), _ptr(value),
+                                  _ptr(a), _ptr(b), _ptr(dt_bias), _ptr(decay_scale),
+                                  _ptr(state_pool), _ptr(actual_seq_lengths),
+                                  _ptr(ssm_state_indices), _ptr(gk),
+                                  _ptr(num_accepted_tokens), float(scale_value), _ptr(out),
+                                  stream)
+    _check(rc)
+    return out, state_pool

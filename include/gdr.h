@@ -1,0 +1,160 @@
+/*
+ * gdr.h - C ABI of libgdr: the recurrent gated-delta-rule decode step on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one defined on the MindSpore Lite API page
+ * "lite_boost.ops.recurrent_gated_delta_rule" (signature; section 算法流程,
+ * steps 1-4; section 参数 for shapes and dtypes; section 返回 for outputs). For
+ * every batch item b, value head h and token t < actual_seq_lengths[b], in
+ * token order:
+ *
+ *   1. decay         S = S * exp(g[b,h,t]) * exp(gk[b,h,t,i])   (row i of D_k)
+ *   2. memory read   kv_mem = S^T k                              (length D_v)
+ *   3. delta update  S = S + k (x) ((v - kv_mem) * beta[b,h,t])
+ *   4. output        o = S^T (q * scale_value), stored as bfloat16
+ *
+ * gdr_gate_fused additionally computes the gate in front of step 1, as the
+ * "com.microsoft.LinearAttentionGate" README defines it (section Description):
+ * g = decay_scale[h] * softplus(a[b,t,h] + dt_bias[h]), beta = sigmoid(b[b,t,h]).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every tensor pointer is DEVICE memory owned by the caller, dense,
+ *           row-major in the shape order given. The library allocates nothing,
+ *           never synchronises, and returns as soon as the work is queued on
+ *           `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *           The current CUDA device must be the one that holds the tensors.
+ * bf16.     gdr_bf16 is the raw bit pattern of an IEEE-style bfloat16.
+ * State.    state_pool is [pool_size, H_v, D_k, D_v] bf16 (row = D_k,
+ *           column = D_v, D_v contiguous); ssm_state_indices[b] names the slot
+ *           item b reads and writes. The pool is updated IN PLACE: the page's
+ *           `state_out` is the same buffer. Slots no item names are untouched.
+ *           The state is carried in fp32 across the tokens of a call and
+ *           rounded to bf16 (round-to-nearest-even) once, after the item's last
+ *           valid token. Slot indices of one call must be distinct (two items
+ *           writing one slot race).
+ * Lengths.  actual_seq_lengths[b] is clamped to [0, T]. Tokens t >= length are
+ *           padding: their inputs are not read, out[b,:,t,:] is +0.0, the state
+ *           does not change. An item whose slot index lies outside
+ *           [0, pool_size) is skipped the same way (all-zero out, no slot
+ *           touched); the library never traps on device values.
+ * Heads.    H_v must be a multiple of H_qk; value head h reads query/key head
+ *           h / (H_v / H_qk) (grouped / multi-query heads).
+ * Aliasing. Inputs must not overlap `out` or `state_pool`.
+ * Sizes.    1 <= T <= 8 (decode only); D_k in {64, 128}; D_v a positive
+ *           multiple of 64; H_qk, H_v, pool_size >= 1; B >= 0 (B == 0 queues
+ *           nothing and returns GDR_OK).
+ * Alignment: query, key, value, gk, state_pool and out must be 16-byte aligned.
+ * Errors.   Every check runs on the host before anything is queued; a failed
+ *           check returns its status and queues nothing. GDR_ERR_CUDA reports a
+ *           launch failure. gdr_last_error() describes the most recent failure
+ *           of the calling thread.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define GDR_API
+#else
+#define GDR_API __attribute__((visibility("default")))
+#endif
+
+/* Raw bfloat16 bits. */
+typedef uint16_t gdr_bf16;
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* gdr_stream_t;
+
+/* Sizes of one call. B batch items, T padded tokens per item, H_qk query/key
+ * heads, H_v value heads, D_k key width (state rows), D_v value width (state
+ * columns), pool_size slots in state_pool. */
+typedef struct gdr_dims {
+  int32_t B;
+  int32_t T;
+  int32_t H_qk;
+  int32_t H_v;
+  int32_t D_k;
+  int32_t D_v;
+  int32_t pool_size;
+} gdr_dims;
+
+typedef enum gdr_status {
+  GDR_OK = 0,
+  GDR_ERR_NULL = 1,        /* a required pointer is NULL */
+  GDR_ERR_DIMS = 2,        /* a size is out of range or inconsistent */
+  GDR_ERR_ALIGN = 3,       /* a tensor is not 16-byte aligned */
+  GDR_ERR_UNSUPPORTED = 4, /* valid sizes this build has no kernel for */
+  GDR_ERR_CUDA = 5         /* the CUDA runtime reported an error */
+} gdr_status;
+
+/*
+ * gdr_decode - one decode call of the op on "lite_boost.ops.recurrent_gated_delta_rule"
+ * (signature and section 算法流程). Argument order follows the page.
+ *
+ *   query               [B, H_qk, T, D_k] bf16  (multiplied by scale_value)
+ *   key                 [B, H_qk, T, D_k] bf16
+ *   value               [B, H_v,  T, D_v] bf16
+ *   beta                [B, H_v,  T]      bf16
+ *   state_pool          [pool_size, H_v, D_k, D_v] bf16, read and written in place
+ *   actual_seq_lengths  [B] int32, valid tokens per item
+ *   ssm_state_indices   [B] int32, pool slot per item
+ *   g                   [B, H_v, T]       fp32
+ *   gk                  [B, H_v, T, D_k]  fp32
+ *   num_accepted_tokens [B] int32 or NULL: accepted for the page's signature;
+ *                       it does not enter the arithmetic and is not read
+ *   scale_value         the page's query scale (1.0 is its default)
+ *   out                 [B, H_v, T, D_v]  bf16, fully written
+ *   stream              CUDA stream the work is queued on
+ *
+ * Returns a gdr_status.
+ */
+GDR_API int gdr_decode(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
+                       const gdr_bf16* value, const gdr_bf16* beta, gdr_bf16* state_pool,
+                       const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
+                       const float* g, const float* gk, const int32_t* num_accepted_tokens,
+                       float scale_value, gdr_bf16* out, gdr_stream_t stream);
+
+/*
+ * gdr_gate_fused - gdr_decode with the LinearAttentionGate computed in the
+ * kernel ("com.microsoft.LinearAttentionGate", sections Description and
+ * Inputs): per token and value head, in fp32,
+ *   g    = decay_scale[h] * softplus(a[b,t,h] + dt_bias[h])
+ *   beta = sigmoid(b[b,t,h])
+ * The gate values stay in fp32 registers; nothing narrows them.
+ *
+ *   a, b         [B, T, H_v] bf16 (heads on the last axis)
+ *   dt_bias      [H_v] fp32
+ *   decay_scale  [H_v] fp32 (for gated DeltaNet, -exp(A_log))
+ * Every other argument is as for gdr_decode; there is no g and no beta.
+ * Returns a gdr_status.
+ */
+GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
+                           const gdr_bf16* value, const gdr_bf16* a, const gdr_bf16* b,
+                           const float* dt_bias, const float* decay_scale, gdr_bf16* state_pool,
+                           const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
+                           const float* gk, const int32_t* num_accepted_tokens,
+                           float scale_value, gdr_bf16* out, gdr_stream_t stream);
+
+/* Static English name of a gdr_status value ("GDR_OK", ...); "unknown status"
+ * for other values. Never NULL. */
+GDR_API const char* gdr_status_string(int status);
+
+/* Description of the most recent failed call made by the calling thread
+ * (which check failed, or the CUDA error string); "" if none failed yet. The
+ * pointer stays valid until the thread's next call into the library. */
+GDR_API const char* gdr_last_error(void);
+
+/* Library ABI version, currently 1. */
+GDR_API int gdr_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */
