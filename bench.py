@@ -225,6 +225,8 @@ def run_gdr(args):
 
     binding.lib()  # fail loudly now if the library is missing
     w = workloads.workload(args.workload)
+    if args.batch is not None:
+        w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch, pool=args.batch)
     gated = w.gated
     # Each rank decodes its own batch: independent sequences and pool slots.
     x = workloads.make_inputs(w, seed=w.seed + 7919 * rank)
@@ -386,6 +388,8 @@ def run_reference(args):
     if rank != 0:
         return  # rank 0 alone times the CPU oracle
     w = workloads.workload(args.workload)
+    if args.batch is not None:
+        w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch, pool=args.batch)
     x = workloads.make_inputs(w)
     n_steps = args.warmup + args.steps
     budget_total = args.reference_seconds
@@ -432,6 +436,9 @@ def main():
     ap.add_argument("--impl", choices=("gdr", "reference"), default="gdr")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     type=lambda s: int(s) if s.isdigit() else s)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B (and the pool size) of the workload, e.g. for a small "
+                         "profiling case of the same kernel")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

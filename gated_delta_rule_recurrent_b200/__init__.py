@@ -8,9 +8,10 @@ fallback).
 """
 from __future__ import annotations
 
-__all__ = ["decode", "decode_gated", "GdrError", "lib", "library_path"]
+__all__ = ["decode", "decode_gated", "device_error", "GdrError", "lib", "library_path"]
 
-_LAZY = {"decode", "decode_gated", "GdrError", "lib", "library_path", "STATUS_NAMES"}
+_LAZY = {"decode", "decode_gated", "device_error", "GdrError", "lib", "library_path",
+         "STATUS_NAMES"}
 
 
 def __getattr__(name):

@@ -15,7 +15,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["decode", "decode_gated", "GdrError", "lib", "library_path", "STATUS_NAMES", "Dims"]
+__all__ = ["decode", "decode_gated", "device_error", "GdrError", "lib", "library_path",
+           "STATUS_NAMES", "Dims"]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.gdr_last_error.restype = ctypes.c_char_p
         L.gdr_abi_version.argtypes = []
         L.gdr_abi_version.restype = ctypes.c_int
+        L.gdr_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+        L.gdr_device_error.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -76,6 +79,16 @@ def lib() -> ctypes.CDLL:
 def _check(rc: int) -> None:
     if rc != 0:
         raise GdrError(rc, lib().gdr_last_error().decode())
+
+
+def device_error(reset: bool = True, device=None) -> int:
+    """The device error word of ``device`` (bit 0: a consumer wait ran out of time,
+    bit 1: a producer wait, bit 2: the final drain). Synchronises the device."""
+    flags = ctypes.c_uint32(0)
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        rc = lib().gdr_device_error(ctypes.byref(flags), int(bool(reset)))
+    _check(rc)
+    return int(flags.value)
 
 
 def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape, device) -> None:

@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(PKG_DIR, "libgdr.so")
 HASH_PATH = LIB_PATH + ".srchash"
 
 SOURCES = [os.path.join(CSRC, "gdr_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "gdr_decode.cuh"), os.path.join(INCLUDE, "gdr.h")]
+DEPS = SOURCES + [os.path.join(CSRC, "gdr_decode.cuh"), os.path.join(CSRC, "gdr_decode_tma.cuh"),
+                  os.path.join(INCLUDE, "gdr.h")]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = [

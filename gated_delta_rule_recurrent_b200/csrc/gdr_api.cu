@@ -4,14 +4,19 @@
 // Everything here runs on the host before any launch. A failed check returns
 // its status with nothing queued; device values (lengths, slot indices) are
 // handled by the kernel without traps.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "gdr.h"
 #include "gdr_decode.cuh"
+#include "gdr_decode_tma.cuh"
 
 namespace {
 
@@ -41,23 +46,196 @@ int check_dims(const gdr_dims* d) {
   // Grid size: B * H_v * (D_v / 64) CTAs must fit a 31-bit grid dimension.
   const long long ctas = static_cast<long long>(d->B) * d->H_v * (d->D_v / gdr::kSliceCols);
   if (ctas > 0x7fffffffLL) return fail(GDR_ERR_DIMS, "B * H_v * D_v / 64 exceeds 2^31 - 1");
+  // TMA row coordinates of the pool are 32-bit signed.
+  if (static_cast<long long>(d->pool_size) * d->H_v * d->D_k > 0x7fffffffLL)
+    return fail(GDR_ERR_UNSUPPORTED, "pool_size * H_v * D_k exceeds 2^31 - 1");
   return GDR_OK;
 }
 
-template <int DK, bool GATED>
-int launch(const gdr::DecodeParams& p, cudaStream_t stream) {
-  const int smem_bytes = gdr::decode_smem_floats<DK>(p.T) * static_cast<int>(sizeof(float));
-  const unsigned grid = static_cast<unsigned>(p.B) * p.H_v * p.n_slices;
-  gdr::decode_kernel<DK, GATED><<<grid, DK, smem_bytes, stream>>>(p);
-  const cudaError_t err = cudaGetLastError();
+// ---------------------------------------------------------------- TMA path
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+#ifndef GDR_MAX_STAGES
+#define GDR_MAX_STAGES 6
+#endif
+constexpr int kMaxStages = GDR_MAX_STAGES;
+
+struct DeviceProps {
+  int sms = 0;
+  int smem_per_sm = 0;
+  int smem_optin = 0;
+};
+
+int device_props(int dev, DeviceProps* out) {
+  static DeviceProps cache[kMaxDevices];
+  static std::atomic<bool> ready[kMaxDevices];
+  if (dev < 0 || dev >= kMaxDevices) return fail(GDR_ERR_CUDA, "device ordinal out of range");
+  if (!ready[dev].load(std::memory_order_acquire)) {
+    DeviceProps p;
+    if (cudaDeviceGetAttribute(&p.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&p.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor,
+                               dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&p.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return fail(GDR_ERR_CUDA, "cudaDeviceGetAttribute failed");
+    cache[dev] = p;
+    ready[dev].store(true, std::memory_order_release);
+  }
+  *out = cache[dev];
+  return GDR_OK;
+}
+
+// Launch shape of one kernel instantiation on one device for one T.
+struct LaunchConfig {
+  int n_stages = 0;
+  int smem = 0;
+  int ctas_per_sm = 0;
+};
+
+template <int DK, int VS, bool GATED>
+int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
+  using Shape = gdr::TmaShape<DK, VS>;
+  static LaunchConfig cache[kMaxDevices][gdr::kMaxT + 1];
+  static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
+  if (ready[dev][T].load(std::memory_order_acquire)) {
+    *out = cache[dev][T];
+    return GDR_OK;
+  }
+  auto kernel = gdr::decode_tma_kernel<DK, VS, GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         props.smem_optin);
+  // All of the unified L1/shared storage as shared memory, so that the CTAs
+  // the stage budget is split for can be co-resident.
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+  cudaFuncAttributes fa;
+  if (err == cudaSuccess) err = cudaFuncGetAttributes(&fa, kernel);
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
+  // CTAs per SM from the register footprint, then the stage count from the
+  // shared-memory budget those CTAs split.
+  const int regs_per_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
+  int ctas = 65536 / (regs_per_warp * (Shape::kThreads / 32));
+  ctas = ctas < 1 ? 1 : (ctas > 4 ? 4 : ctas);
+  LaunchConfig c;
+  for (; ctas >= 1; --ctas) {
+    const int stage_bytes = gdr::stage_layout<DK, VS>(T).bytes;
+    const int budget = props.smem_per_sm / ctas - 1024;
+    int n = (budget - 1024 - gdr::cta_extra_bytes<DK, VS>(kMaxStages)) / stage_bytes;
+    n = n > kMaxStages ? kMaxStages : n;
+    if (n < gdr::kMinStages) n = gdr::kMinStages;
+    const int smem = gdr::tma_smem_bytes<DK, VS>(T, n);
+    if (smem > props.smem_optin) continue;
+    // A persistent grid must be co-resident: trust the occupancy calculator.
+    int resident = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, Shape::kThreads, smem);
+    if (err != cudaSuccess)
+      return fail(GDR_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(err));
+    if (resident < 1) continue;
+    c.n_stages = n;
+    c.smem = smem;
+    c.ctas_per_sm = resident < ctas ? resident : ctas;
+    break;
+  }
+  if (c.ctas_per_sm == 0) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+  cache[dev][T] = c;
+  ready[dev][T].store(true, std::memory_order_release);
+  *out = c;
+  return GDR_OK;
+}
+
+template <int DK, int VS, bool GATED>
+int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
+  using Shape = gdr::TmaShape<DK, VS>;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
+  DeviceProps props;
+  int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  LaunchConfig cfg;
+  rc = launch_config<DK, VS, GATED>(dev, p.T, props, &cfg);
+  if (rc != GDR_OK) return rc;
+  const int n_stages = cfg.n_stages;
+  const int smem = cfg.smem;
+  const int ctas_per_sm = cfg.ctas_per_sm;
+
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  // The pool seen as a 2-D bf16 matrix: rows = pool * H_v * D_k, columns = D_v.
+  CUtensorMap map;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(p.D_v),
+                              static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(p.D_v) * 2};
+  const cuuint32_t box[2] = {VS, DK};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                             const_cast<uint16_t*>(p.state_pool), gdim, gstride, box, estride,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+
+  const int n_tiles = p.B * p.H_v * (p.D_v / VS);
+  const int max_ctas = ctas_per_sm * props.sms;
+  const int grid = n_tiles < max_ctas ? n_tiles : max_ctas;
+  gdr::decode_tma_kernel<DK, VS, GATED><<<grid, Shape::kThreads, smem, stream>>>(map, p, n_tiles,
+                                                                                 n_stages);
+  err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
   return GDR_OK;
 }
 
+// State elements per tile the slice width aims at (D_k x slice).
+#ifndef GDR_TILE_ELEMS
+#define GDR_TILE_ELEMS 16384
+#endif
+
+// Column-slice width: at most GDR_TILE_ELEMS / D_k columns, the widest such
+// width that divides D_v and still gives every SM two tiles, else the
+// narrowest width that divides D_v.
+int pick_slice(int D_k, int D_v, long long items_heads, int sms) {
+  const int widths[3] = {256, 128, 64};
+  int narrowest = 64;
+  for (int i = 0; i < 3; ++i) {
+    if (widths[i] * D_k > GDR_TILE_ELEMS || (D_k == 128 && widths[i] > 128)) continue;
+    if (D_v % widths[i] != 0) continue;
+    narrowest = widths[i];
+    if (items_heads * (D_v / widths[i]) >= 2LL * sms) return widths[i];
+  }
+  return narrowest;
+}
+
 int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, cudaStream_t stream) {
-  if (D_k == 64) return gated ? launch<64, true>(p, stream) : launch<64, false>(p, stream);
-  return gated ? launch<128, true>(p, stream) : launch<128, false>(p, stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
+  DeviceProps props;
+  const int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  const int vs = pick_slice(D_k, p.D_v, static_cast<long long>(p.B) * p.H_v, props.sms);
+  if (D_k == 64) {
+    if (vs == 256) return gated ? launch_tma<64, 256, true>(p, stream) : launch_tma<64, 256, false>(p, stream);
+    if (vs == 128) return gated ? launch_tma<64, 128, true>(p, stream) : launch_tma<64, 128, false>(p, stream);
+    return gated ? launch_tma<64, 64, true>(p, stream) : launch_tma<64, 64, false>(p, stream);
+  }
+  if (vs == 128) return gated ? launch_tma<128, 128, true>(p, stream) : launch_tma<128, 128, false>(p, stream);
+  return gated ? launch_tma<128, 64, true>(p, stream) : launch_tma<128, 64, false>(p, stream);
 }
 
 gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gdr_bf16* key,
@@ -158,6 +336,20 @@ GDR_API const char* gdr_status_string(int status) {
 }
 
 GDR_API const char* gdr_last_error(void) { return g_last_error.c_str(); }
+
+GDR_API int gdr_device_error(uint32_t* flags, int reset) {
+  if (flags == nullptr) return fail(GDR_ERR_NULL, "flags is NULL");
+  unsigned int v = 0;
+  cudaError_t err = cudaMemcpyFromSymbol(&v, gdr::g_device_error, sizeof(v));
+  if (err == cudaSuccess && reset) {
+    const unsigned int zero = 0;
+    err = cudaMemcpyToSymbol(gdr::g_device_error, &zero, sizeof(zero));
+  }
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("reading the device error word: ") + cudaGetErrorString(err));
+  *flags = v;
+  return GDR_OK;
+}
 
 GDR_API int gdr_abi_version(void) { return 1; }
 

@@ -150,6 +150,16 @@ GDR_API const char* gdr_status_string(int status);
  * pointer stays valid until the thread's next call into the library. */
 GDR_API const char* gdr_last_error(void);
 
+/* Device-side error word of the current device, OR-ed over every kernel run
+ * since the last reset: bit 0 = a consumer wait on staged data ran out of time,
+ * bit 1 = the producer's wait for a free stage ran out of time, bit 2 = the
+ * final wait for in-flight copies ran out of time. A wait that runs out never
+ * hangs the kernel: it flags the word and the kernel finishes, and the outputs
+ * of that call are invalid. Writes the word to *flags and clears it when
+ * `reset` is nonzero. SYNCHRONISES the device (a blocking copy). No
+ * counterpart on the pages: every bounded wait of the kernels reports here. */
+GDR_API int gdr_device_error(uint32_t* flags, int reset);
+
 /* Library ABI version, currently 1. */
 GDR_API int gdr_abi_version(void);
 

@@ -68,6 +68,22 @@ def test_ragged_shapes(D_k, D_v, H_qk, H_v, T, gated):
     _roundtrip(workloads.make_inputs(w, poison_padding=True), gated)
 
 
+@pytest.mark.parametrize("gated", [False, True])
+def test_many_tiles_with_empty_items(gated):
+    """Thousands of tiles per call, so every CTA reuses its stages many times,
+    with runs of zero-length items and slots outside the pool between stored tiles."""
+    w = workloads.WORKLOADS[3].replace(name="sparse", B=96, pool=128, seed=4242)
+    x = workloads.make_inputs(w, poison_padding=True)
+    L = x["actual_seq_lengths"]
+    L[1::3] = 0
+    L[2::7] = -1
+    x["ssm_state_indices"][5::11] = 1000
+    x["num_accepted_tokens"] = L.clamp(0, 8)
+    for name in ("query", "key", "value", "gk"):
+        x[name][L <= 0] = float("nan")
+    _roundtrip(x, gated)
+
+
 @pytest.mark.parametrize("T", list(range(1, 9)))
 def test_every_token_count(T):
     w = workloads.WORKLOADS[0].replace(name=f"T{T}", B=3, T=T, pool=4, lengths="full",
@@ -138,6 +154,15 @@ def test_side_stream_and_determinism():
     torch.cuda.synchronize()
     assert np.array_equal(bits(out1), bits(out2))
     assert np.array_equal(bits(pool1), bits(pool2))
+
+
+def test_device_error_word_stays_clear():
+    from gated_delta_rule_recurrent_b200 import device_error
+
+    device_error(reset=True)
+    for cfg in (0, 2, 3):
+        _roundtrip(workloads.make_inputs(cfg), cfg == 2)
+    assert device_error(reset=True) == 0
 
 
 def test_device_errors_reported_without_launch():
