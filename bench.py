@@ -42,6 +42,7 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 DEFAULT_WORKLOAD = 4
 KERNEL_SOURCE_FILES = ("gated_delta_rule_recurrent_b200/csrc/gdr_decode.cuh",
+                       "gated_delta_rule_recurrent_b200/csrc/gdr_decode_tma.cuh",
                        "gated_delta_rule_recurrent_b200/csrc/gdr_api.cu")
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gated_B512_H64_64x512_dram.txt")
 
@@ -370,7 +371,7 @@ def run_gdr(args):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth",
-            "kernel": "gdr::decode_kernel", "kernel_ms": kernel_ms,
+            "kernel": "gdr::decode_tma_kernel", "kernel_ms": kernel_ms,
             "bytes_per_launch": step_bytes, "traffic": recorded_traffic(),
         },
         "e2e": e2e,

@@ -106,16 +106,16 @@ struct LaunchConfig {
   int ctas_per_sm = 0;
 };
 
-template <int DK, int VS, bool GATED>
+template <int DK, int VS, int R, bool GATED, bool ONE>
 int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
-  using Shape = gdr::TmaShape<DK, VS>;
+  using Shape = gdr::TmaShape<DK, VS, R>;
   static LaunchConfig cache[kMaxDevices][gdr::kMaxT + 1];
   static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
   if (ready[dev][T].load(std::memory_order_acquire)) {
     *out = cache[dev][T];
     return GDR_OK;
   }
-  auto kernel = gdr::decode_tma_kernel<DK, VS, GATED>;
+  auto kernel = gdr::decode_tma_kernel<DK, VS, R, GATED, ONE>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          props.smem_optin);
   // All of the unified L1/shared storage as shared memory, so that the CTAs
@@ -134,12 +134,12 @@ int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
   ctas = ctas < 1 ? 1 : (ctas > 4 ? 4 : ctas);
   LaunchConfig c;
   for (; ctas >= 1; --ctas) {
-    const int stage_bytes = gdr::stage_layout<DK, VS>(T).bytes;
+    const int stage_bytes = gdr::stage_layout<DK, VS, R, ONE>(T).bytes;
     const int budget = props.smem_per_sm / ctas - 1024;
-    int n = (budget - 1024 - gdr::cta_extra_bytes<DK, VS>(kMaxStages)) / stage_bytes;
+    int n = (budget - 1024 - gdr::cta_extra_bytes<DK, VS, R, ONE>(kMaxStages)) / stage_bytes;
     n = n > kMaxStages ? kMaxStages : n;
     if (n < gdr::kMinStages) n = gdr::kMinStages;
-    const int smem = gdr::tma_smem_bytes<DK, VS>(T, n);
+    const int smem = gdr::tma_smem_bytes<DK, VS, R, ONE>(T, n);
     if (smem > props.smem_optin) continue;
     // A persistent grid must be co-resident: trust the occupancy calculator.
     int resident = 0;
@@ -159,9 +159,9 @@ int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
   return GDR_OK;
 }
 
-template <int DK, int VS, bool GATED>
+template <int DK, int VS, int R, bool GATED, bool ONE>
 int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
-  using Shape = gdr::TmaShape<DK, VS>;
+  using Shape = gdr::TmaShape<DK, VS, R>;
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
@@ -169,7 +169,7 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   LaunchConfig cfg;
-  rc = launch_config<DK, VS, GATED>(dev, p.T, props, &cfg);
+  rc = launch_config<DK, VS, R, GATED, ONE>(dev, p.T, props, &cfg);
   if (rc != GDR_OK) return rc;
   const int n_stages = cfg.n_stages;
   const int smem = cfg.smem;
@@ -177,14 +177,18 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
 
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  // The pool seen as a 2-D bf16 matrix: rows = pool * H_v * D_k, columns = D_v.
+  // The pool seen as a 3-D bf16 array: [pool * H_v * D_k rows][D_v / C blocks][C
+  // columns] with C = min(VS, 256), so one box {C, VS / C, D_k} is a whole tile
+  // and, for VS = D_v, one contiguous (slot, head) state.
   CUtensorMap map;
-  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(p.D_v),
+  constexpr int C = Shape::kBoxCols;
+  const cuuint64_t gdim[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(p.D_v / C),
                               static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK};
-  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(p.D_v) * 2};
-  const cuuint32_t box[2] = {VS, DK};
-  const cuuint32_t estride[2] = {1, 1};
-  const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(C) * 2,
+                                 static_cast<cuuint64_t>(p.D_v) * 2};
+  const cuuint32_t box[3] = {C, Shape::kBoxParts, DK};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                              const_cast<uint16_t*>(p.state_pool), gdim, gstride, box, estride,
                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -194,7 +198,7 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   const int n_tiles = p.B * p.H_v * (p.D_v / VS);
   const int max_ctas = ctas_per_sm * props.sms;
   const int grid = n_tiles < max_ctas ? n_tiles : max_ctas;
-  gdr::decode_tma_kernel<DK, VS, GATED><<<grid, Shape::kThreads, smem, stream>>>(map, p, n_tiles,
+  gdr::decode_tma_kernel<DK, VS, R, GATED, ONE><<<grid, Shape::kThreads, smem, stream>>>(map, p, n_tiles,
                                                                                  n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
@@ -202,40 +206,67 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   return GDR_OK;
 }
 
-// State elements per tile the slice width aims at (D_k x slice).
-#ifndef GDR_TILE_ELEMS
-#define GDR_TILE_ELEMS 16384
-#endif
+using LaunchFn = int (*)(const gdr::DecodeParams&, cudaStream_t);
+struct SliceKernel {
+  int vs;
+  LaunchFn launch;
+};
 
-// Column-slice width: at most GDR_TILE_ELEMS / D_k columns, the widest such
-// width that divides D_v and still gives every SM two tiles, else the
-// narrowest width that divides D_v.
-int pick_slice(int D_k, int D_v, long long items_heads, int sms) {
-  const int widths[3] = {256, 128, 64};
-  int narrowest = 64;
-  for (int i = 0; i < 3; ++i) {
-    if (widths[i] * D_k > GDR_TILE_ELEMS || (D_k == 128 && widths[i] > 128)) continue;
-    if (D_v % widths[i] != 0) continue;
-    narrowest = widths[i];
-    if (items_heads * (D_v / widths[i]) >= 2LL * sms) return widths[i];
+// Tile widths per path, widest first, with the rows each consumer thread
+// holds. The thread count of a block caps the registers ptxas may give a
+// thread (255 up to 256 threads, 168 up to 384, 128 up to 512, 96 up to 640).
+// A single-token call keeps no state in registers (about 75 of them), so a
+// full-width 64 x 512 tile can use 16 consumer warps. A multi-token call keeps
+// fp32 state across tokens and stays within 168 (D_k = 64, 8 rows) or 255
+// (D_k = 128, 16 rows) registers.
+template <bool GATED>
+const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
+  static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED, true>},
+                                        {256, launch_tma<64, 256, 8, GATED, true>},
+                                        {128, launch_tma<64, 128, 8, GATED, true>},
+                                        {64, launch_tma<64, 64, 8, GATED, true>}};
+  static const SliceKernel k128_one[] = {{256, launch_tma<128, 256, 16, GATED, true>},
+                                         {128, launch_tma<128, 128, 16, GATED, true>},
+                                         {64, launch_tma<128, 64, 16, GATED, true>}};
+  static const SliceKernel k64_many[] = {{256, launch_tma<64, 256, 8, GATED, false>},
+                                         {128, launch_tma<64, 128, 8, GATED, false>},
+                                         {64, launch_tma<64, 64, 8, GATED, false>}};
+  static const SliceKernel k128_many[] = {{128, launch_tma<128, 128, 16, GATED, false>},
+                                          {64, launch_tma<128, 64, 16, GATED, false>}};
+  if (D_k == 64) {
+    *n = one ? 4 : 3;
+    return one ? k64_one : k64_many;
   }
-  return narrowest;
+  *n = one ? 3 : 2;
+  return one ? k128_one : k128_many;
 }
 
+// Column-slice width: the widest width that divides D_v and still gives every
+// SM a tile, else the narrowest one; a width whose stage ring does not fit in
+// shared memory (long T) falls back to the next narrower one.
 int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
   DeviceProps props;
-  const int rc = device_props(dev, &props);
+  int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
-  const int vs = pick_slice(D_k, p.D_v, static_cast<long long>(p.B) * p.H_v, props.sms);
-  if (D_k == 64) {
-    if (vs == 256) return gated ? launch_tma<64, 256, true>(p, stream) : launch_tma<64, 256, false>(p, stream);
-    if (vs == 128) return gated ? launch_tma<64, 128, true>(p, stream) : launch_tma<64, 128, false>(p, stream);
-    return gated ? launch_tma<64, 64, true>(p, stream) : launch_tma<64, 64, false>(p, stream);
+  int n = 0;
+  const bool one = p.T == 1;
+  const SliceKernel* ks =
+      gated ? slice_kernels<true>(D_k, one, &n) : slice_kernels<false>(D_k, one, &n);
+  int first = -1;
+  for (int i = 0; i < n; ++i) {
+    if (p.D_v % ks[i].vs != 0) continue;
+    first = i;
+    if (static_cast<long long>(p.B) * p.H_v * (p.D_v / ks[i].vs) >= props.sms) break;
   }
-  if (vs == 128) return gated ? launch_tma<128, 128, true>(p, stream) : launch_tma<128, 128, false>(p, stream);
-  return gated ? launch_tma<128, 64, true>(p, stream) : launch_tma<128, 64, false>(p, stream);
+  if (first < 0) return fail(GDR_ERR_UNSUPPORTED, "no tile width divides D_v");
+  for (int i = first; i < n; ++i) {
+    if (p.D_v % ks[i].vs != 0) continue;
+    rc = ks[i].launch(p, stream);
+    if (rc != GDR_ERR_UNSUPPORTED) return rc;
+  }
+  return rc;
 }
 
 gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gdr_bf16* key,
@@ -259,7 +290,6 @@ gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gd
   p.D_v = d->D_v;
   p.pool_size = d->pool_size;
   p.group = d->H_v / d->H_qk;
-  p.n_slices = d->D_v / gdr::kSliceCols;
   return p;
 }
 

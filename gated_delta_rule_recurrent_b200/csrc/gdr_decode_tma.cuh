@@ -4,33 +4,33 @@
 // (MindSpore Lite API page, section 算法流程) and, when GATED, the gate of
 // "com.microsoft.LinearAttentionGate" (README, section Description).
 //
-// Data flow. A tile is one (item b, value head h, VS-column slice of D_v) block
-// of the state: DK rows x VS bf16 columns of slot ssm_state_indices[b]. Each
-// CTA walks tiles tile = blockIdx.x, + gridDim.x, ... through a ring of
-// shared-memory stages, with three roles:
+// A tile is one (item b, value head h, VS-column slice of D_v) block of the
+// state: all D_k rows x VS bf16 columns of slot ssm_state_indices[b]; with
+// VS = D_v it is the slot's whole contiguous head state. Each CTA walks tiles
+// tile = blockIdx.x, + gridDim.x, ... through a ring of shared-memory stages,
+// with three roles:
 //
-//   producer warp - starts the asynchronous copies of a tile (a 2-D TMA load
-//           of the state box; 1-D bulk copies of the value rows and of the k,
-//           q and gk rows of the valid tokens; 4-byte cp.async copies of the
+//   producer warp - starts the asynchronous copies of a tile (one TMA box for
+//           the state; 1-D bulk copies of the value rows and of the k, q and
+//           gk rows of the valid tokens; 4-byte cp.async copies of the
 //           per-token gate scalars) and, kLookahead tiles later, once they
 //           have landed ("raw" barrier), turns them into what the consumers
 //           use: exp(g + gk) per row (written over gk), k.(q*scale) and beta
 //           per token ("full" barrier). No lane waits on global-memory latency.
-//   consumer warps - keep an 8x8 sub-tile in fp32 registers for all valid
-//           tokens: decay in place; the column sums kv_mem = S^T k and
-//           p = S^T q together; one CTA barrier per token to combine partial
-//           sums across warps; delta; output o = scale * p +
-//           delta * (k.q*scale), which is step 4's S_new^T (q*scale) with the
-//           sums reordered; rank-1 update. Once done reading the input stage
-//           they give it back to the producer ("empty" barrier), then write
-//           the new tile as bf16 into a separate output buffer ("out_full").
-//   storer warp - issues the TMA store of every output buffer and frees the
-//           buffer ("out_empty") once the store has read it.
+//   consumer warps - each owns ALL D_k rows of a band of 32 columns; lane
+//           (row lane 0..7, column lane 0..3) holds D_k/8 rows x 8 columns in
+//           fp32 registers for all valid tokens. Every reduction over D_k is a
+//           warp shuffle, so consumer warps never synchronise with each other
+//           and drift apart freely. Per token: decay in place; the column sums
+//           kv_mem = S^T k and p = S^T q together; a reduce-scatter over the
+//           row lanes; delta; output o = scale * p + delta * (k.q*scale),
+//           which is step 4's S_new^T (q*scale) with the sums reordered;
+//           rank-1 update. A warp gives the stage back ("empty" barrier) as
+//           soon as it has read what it needs, and then streams its rows of the
+//           new state to the pool from registers with 16-byte stores.
 //
-// Input stages therefore cycle at the pace of HBM latency plus compute; the
-// store drain only holds the small output ring.
-//
-// HBM sees one bulk read and one bulk write of every touched state tile.
+// HBM sees one bulk read and one write of every touched state tile, and a
+// stage is held only while its tile is loaded and computed.
 //
 // Every mbarrier wait is bounded (a clock budget of a few seconds). A wait
 // that runs out sets a bit in a device-global error word and the kernel goes
@@ -51,7 +51,6 @@ namespace gdr {
 constexpr unsigned kErrConsumerWait = 1u;
 constexpr unsigned kErrProducerWait = 2u;
 constexpr unsigned kErrDrainWait = 4u;
-constexpr unsigned kErrStorerWait = 8u;
 
 static __device__ unsigned int g_device_error = 0;
 
@@ -59,69 +58,68 @@ constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
 // Tuning constants (compile-time; the defaults are the measured best).
 #ifndef GDR_LOOKAHEAD
-#define GDR_LOOKAHEAD 2
-#endif
-#ifndef GDR_STORES_IN_FLIGHT
-#define GDR_STORES_IN_FLIGHT 1
+#define GDR_LOOKAHEAD 1
 #endif
 // The producer finalises tile j - kLookahead after starting the copies of tile j.
 constexpr int kLookahead = GDR_LOOKAHEAD;
-// TMA stores whose shared-memory reads may still be pending before the
-// storer frees their output buffers.
-constexpr int kStoresInFlight = GDR_STORES_IN_FLIGHT;
-// Neither ring may wait on itself: the producer refills a stage only after the
-// consumers finished its previous tile, which the producer finalised
-// kLookahead issues later; an output buffer is freed one stored tile late.
+// The ring never waits on itself: the producer refills a stage only after the
+// consumers finished the tile it held, which the producer finalised kLookahead
+// issues after starting it.
 constexpr int kMinStages = kLookahead + 1;
-constexpr int kOutBuffers = kStoresInFlight + 1;
-static_assert(kStoresInFlight >= 1 && kStoresInFlight <= 4, "release queue holds 1..4 stages");
 
-template <int DK, int VS>
+// R: state rows per thread (8 or 16); a lane always holds 8 columns.
+template <int DK, int VS, int R>
 struct TmaShape {
-  static constexpr int kRows = 8;              // state rows per thread
-  static constexpr int kWarpRows = 4 * kRows;  // a warp covers 32 rows x 64 columns
-  static constexpr int kWC = VS / 64;          // warp columns
-  static constexpr int kWR = DK / kWarpRows;   // warp rows
-  static constexpr int kConsumerWarps = kWC * kWR;
+  static constexpr int kRows = R;
+  static constexpr int kRowLanes = DK / kRows;      // lanes that split the D_k rows: 4, 8 or 16
+  static constexpr int kColLanes = 32 / kRowLanes;  // lanes that split the band: 8, 4 or 2
+  static constexpr int kWarpCols = kColLanes * 8;   // columns per consumer warp: 64, 32 or 16
+  static constexpr int kConsumerWarps = VS / kWarpCols;
   static constexpr int kConsumers = kConsumerWarps * 32;
-  static constexpr int kThreads = kConsumers + 64;  // + producer warp + storer warp
+  static constexpr int kThreads = kConsumers + 32;  // + the producer warp
   static constexpr int kStateBytes = DK * VS * 2;
+  static constexpr int kBoxCols = VS < 256 ? VS : 256;  // TMA box extents: columns,
+  static constexpr int kBoxParts = VS / kBoxCols;       // column blocks, rows (= D_k)
+  static_assert(DK == 64 || DK == 128, "D_k must be 64 or 128");
+  static_assert(R == 8 || R == 16, "8 or 16 rows per thread");
+  static_assert(kRowLanes >= 4 && kRowLanes <= 16, "4 to 16 row lanes");
+  static_assert(VS % kWarpCols == 0 && kConsumerWarps >= 1 && kConsumerWarps <= 16,
+                "one to sixteen consumer warps per tile");
 };
 
 // Byte offsets inside one stage, for T padded tokens.
 struct StageLayout {
-  int v, k, q, sd, raw, beta, kq, meta, bytes;
+  int v, k, q, gk, rv, raw, beta, kq, meta, bytes;
 };
 
-template <int DK, int VS>
+// ONE (single-token calls): the producer also writes float4 row vectors
+// {d k, d q_s, d, k}; multi-token calls use the compact form, d written over gk.
+template <int DK, int VS, int R, bool ONE>
 __host__ __device__ inline StageLayout stage_layout(int T) {
   StageLayout s;
-  s.v = TmaShape<DK, VS>::kStateBytes;  // bf16 [T][VS]   value rows of the slice
+  s.v = TmaShape<DK, VS, R>::kStateBytes;  // bf16 [T][VS]   value rows of the slice
   s.k = s.v + T * VS * 2;               // bf16 [T][DK]   key rows
   s.q = s.k + T * DK * 2;               // bf16 [T][DK]   query rows
-  s.sd = s.q + T * DK * 2;              // fp32 [T][DK]   gk, then exp(g + gk)
-  s.raw = s.sd + T * DK * 4;            // u32 [2][8]     gate scalar words
+  s.gk = s.q + T * DK * 2;              // fp32 [T][DK]   gk rows (multi-token: then d = exp(g + gk))
+  s.rv = s.gk + T * DK * 4;             // fp32x4 [T][DK] {d*k, d*q*scale, d, k} (single-token only)
+  s.raw = s.rv + (ONE ? T * DK * 16 : 0);  // u32 [2][8]  gate scalar words
   s.beta = s.raw + 64;                  // fp32 [8]
   s.kq = s.beta + 32;                   // fp32 [8]       k . (q * scale)
-  s.meta = s.kq + 32;                   // int32 [4]      length, slot, consumer failure
+  s.meta = s.kq + 32;                   // int32 [4]      length, slot
   s.bytes = (s.meta + 16 + 1023) & ~1023;
   return s;
 }
 
-// CTA-level area after the input stages: kOutBuffers output tiles with their
-// (length, slot, failure) words, two buffers of per-warp partial sums, and the
-// mbarriers (three per input stage, two per output buffer).
-template <int DK, int VS>
+// CTA-level area after the stages: three mbarriers per stage.
+template <int DK, int VS, int R, bool ONE>
 __host__ __device__ inline int cta_extra_bytes(int n_stages) {
-  using S = TmaShape<DK, VS>;
-  return kOutBuffers * S::kStateBytes + kOutBuffers * 16 + 2 * S::kConsumerWarps * 32 * 4 * 4 +
-         (3 * n_stages + 2 * kOutBuffers) * 8;
+  return 3 * n_stages * 8;
 }
 
-template <int DK, int VS>
+template <int DK, int VS, int R, bool ONE>
 __host__ __device__ inline int tma_smem_bytes(int T, int n_stages) {
-  return 1024 /* alignment slack */ + n_stages * stage_layout<DK, VS>(T).bytes +
-         cta_extra_bytes<DK, VS>(n_stages);
+  return 1024 /* alignment slack */ + n_stages * stage_layout<DK, VS, R, ONE>(T).bytes +
+         cta_extra_bytes<DK, VS, R, ONE>(n_stages);
 }
 
 // ---------------------------------------------------------------- PTX helpers
@@ -170,12 +168,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
   return true;
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar) {
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(map), "r"(x), "r"(y), "r"(bar)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
 }
 
@@ -197,48 +195,6 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
 // Arrive on `bar` once every cp.async this thread has issued so far has landed.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::
-                   "l"(map),
-               "r"(x), "r"(y), "r"(src)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// Barrier over `n` threads that also returns the AND of `v` over them.
-__device__ __forceinline__ bool named_bar_and(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
 }
 
 __device__ __forceinline__ void flag_error(unsigned bit) { atomicOr(&g_device_error, bit); }
@@ -285,20 +241,21 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 w, float (&f)[8]) {
 
 // ---------------------------------------------------------------- the kernel
 
-constexpr int kConsumerBar = 1;  // named barrier of the consumer warps
-
-template <int DK, int VS, bool GATED>
-__global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
+// ONE: the call has a single token (T = 1), the common decode case; the
+// consumers then keep only bf16 state words between the two passes.
+template <int DK, int VS, int RR, bool GATED, bool ONE>
+__global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     decode_tma_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                       const int n_tiles, const int n_stages) {
-  using Shape = TmaShape<DK, VS>;
-  constexpr int NC = Shape::kConsumers;
+  using Shape = TmaShape<DK, VS, RR>;
   constexpr int CW = Shape::kConsumerWarps;
-  constexpr int WC = Shape::kWC;
-  constexpr int WR = Shape::kWR;
   constexpr int R = Shape::kRows;
+  constexpr int RL = Shape::kRowLanes;
+  constexpr int CL = Shape::kColLanes;
+  constexpr int WCOLS = Shape::kWarpCols;
+  constexpr int NV = 16 / RL;  // reduced values per lane after the reduce-scatter: 4, 2 or 1
   const int T = p.T;
-  const StageLayout lay = stage_layout<DK, VS>(T);
+  const StageLayout lay = stage_layout<DK, VS, RR, ONE>(T);
 
   // Stages start on a 1024-byte boundary of the shared window. The offset is
   // added to the __shared__ array itself so every access stays a shared-memory
@@ -306,15 +263,10 @@ __global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_base = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
-  uint8_t* obuf = smem + n_stages * lay.bytes;                         // [kOut][DK][VS] bf16
-  int* ometa = reinterpret_cast<int*>(obuf + kOutBuffers * Shape::kStateBytes);  // [kOut][4]
-  float* red = reinterpret_cast<float*>(ometa + 4 * kOutBuffers);         // [2][CW][32][4]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * CW * 128);
-  const uint32_t raw0 = smem_addr(bars);             // copies landed
-  const uint32_t full0 = raw0 + 8 * n_stages;        // producer finished the stage
-  const uint32_t empty0 = full0 + 8 * n_stages;      // consumers done reading the stage
-  const uint32_t ofull0 = empty0 + 8 * n_stages;     // consumers wrote the output buffer
-  const uint32_t oempty0 = ofull0 + 8 * kOutBuffers;  // the store has read the buffer
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + n_stages * lay.bytes);
+  const uint32_t raw0 = smem_addr(bars);         // copies landed
+  const uint32_t full0 = raw0 + 8 * n_stages;    // producer finished the stage
+  const uint32_t empty0 = full0 + 8 * n_stages;  // consumers are done reading the stage
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -325,13 +277,9 @@ __global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < n_stages; ++i) {
-      mbar_init(raw0 + 8 * i, 32);  // one cp.async arrival per producer lane
+      mbar_init(raw0 + 8 * i, 32);    // one cp.async arrival per producer lane
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, CW);  // one arrival per consumer warp
-    }
-    for (int i = 0; i < kOutBuffers; ++i) {
-      mbar_init(ofull0 + 8 * i, CW);
-      mbar_init(oempty0 + 8 * i, 1);
     }
     fence_mbar_init();
   }
@@ -383,12 +331,13 @@ __global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
           meta[1] = s;
           if (L > 0) {
             mbar_expect_tx(rawb, Shape::kStateBytes + L * (VS * 2 + DK * 8));
-            tma_load_2d(smem_addr(st), &pool_map, col0, (s * p.H_v + h) * DK, rawb);
+            tma_load_3d(smem_addr(st), &pool_map, 0, col0 / Shape::kBoxCols,
+                        (s * p.H_v + h) * DK, rawb);
             const size_t qk_off = (static_cast<size_t>(b) * p.H_qk + hq) * T * DK;
             const size_t gk_off = (static_cast<size_t>(b) * p.H_v + h) * T * DK;
             bulk_load(smem_addr(st + lay.k), p.key + qk_off, L * DK * 2, rawb);
             bulk_load(smem_addr(st + lay.q), p.query + qk_off, L * DK * 2, rawb);
-            bulk_load(smem_addr(st + lay.sd), p.gk + gk_off, L * DK * 4, rawb);
+            bulk_load(smem_addr(st + lay.gk), p.gk + gk_off, L * DK * 4, rawb);
             const uint16_t* vsrc =
                 p.value + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + col0;
             for (int t = 0; t < L; ++t)
@@ -432,7 +381,8 @@ __global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
         const uint32_t* rawv = reinterpret_cast<const uint32_t*>(st + lay.raw);
         float* sbeta = reinterpret_cast<float*>(st + lay.beta);
         float* skq = reinterpret_cast<float*>(st + lay.kq);
-        float* sd = reinterpret_cast<float*>(st + lay.sd);
+        float* sgk = reinterpret_cast<float*>(st + lay.gk);
+        float4* srv = reinterpret_cast<float4*>(st + lay.rv);
         const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);
         const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
         float dtb = 0.0f, dsc = 0.0f;
@@ -461,14 +411,21 @@ __global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const int i = lane + 32 * e;
-            sd[t * DK + i] = expf(gt + sd[t * DK + i]);  // exp(g) * exp(gk) as one exponential
-            kq = fmaf(bf16_bits_to_f32(sk[t * DK + i]), bf16_bits_to_f32(sq[t * DK + i]), kq);
+            const float d = expf(gt + sgk[t * DK + i]);  // exp(g) * exp(gk) as one exponential
+            const float kv = bf16_bits_to_f32(sk[t * DK + i]);
+            const float qs = bf16_bits_to_f32(sq[t * DK + i]) * p.scale;
+            if constexpr (ONE) {
+              srv[t * DK + i] = make_float4(d * kv, d * qs, d, kv);
+            } else {
+              sgk[t * DK + i] = d;
+            }
+            kq = fmaf(kv, qs, kq);
           }
           kq = warp_sum(kq);
           __syncwarp();
           if (lane == 0) {
             sbeta[t] = bt;
-            skq[t] = kq * p.scale;
+            skq[t] = kq;  // k . (q * scale)
           }
         }
         __syncwarp();
@@ -486,259 +443,273 @@ __global__ void __launch_bounds__(TmaShape<DK, VS>::kThreads, 1)
     return;
   }
 
-  if (warp == CW + 1) {
-    // ================================================================ storer
-    if (lane != 0) return;
-    // Output buffers whose TMA stores may still be reading them, oldest first.
-    int pend[kStoresInFlight + 1] = {};
-    int n_pend = 0;
-    for (int it = 0; it < n_mine; ++it) {
-      const int tile = blockIdx.x + it * gridDim.x;
-      const int slice = tile % n_slices;
-      const int h = (tile / n_slices) % p.H_v;
-      const int ob = it % kOutBuffers;
-      const uint32_t phase = (it / kOutBuffers) & 1;
-      const bool ok = mbar_wait_bounded(ofull0 + 8 * ob, phase);
-      if (!ok) flag_error(kErrStorerWait);
-      const int L = ometa[4 * ob + 0];
-      const int s = ometa[4 * ob + 1];
-      if (ok && ometa[4 * ob + 2] == 0 && L > 0 && s >= 0 && s < p.pool_size) {
-        tma_store_2d(&pool_map, slice * VS, (s * p.H_v + h) * DK,
-                     smem_addr(obuf + ob * Shape::kStateBytes));
-        bulk_commit();
-#pragma unroll
-        for (int q = 0; q <= kStoresInFlight; ++q)
-          if (q == n_pend) pend[q] = ob;  // constant indices keep pend in registers
-        ++n_pend;
-        if (n_pend > kStoresInFlight) {
-          // all but the newest kStoresInFlight stores have read their buffers
-          bulk_wait_read<kStoresInFlight>();
-          mbar_arrive(oempty0 + 8 * pend[0]);
-#pragma unroll
-          for (int q = 0; q < kStoresInFlight; ++q) pend[q] = pend[q + 1];
-          --n_pend;
-        }
-      } else {
-        // Nothing to store from this buffer. Free it, and every pending one
-        // once its store has read it, so no buffer waits on a later store.
-        bulk_wait_read<0>();
-#pragma unroll
-        for (int q = 0; q < kStoresInFlight; ++q)
-          if (q < n_pend) mbar_arrive(oempty0 + 8 * pend[q]);
-        n_pend = 0;
-        mbar_arrive(oempty0 + 8 * ob);
-      }
-    }
-    bulk_wait_all();
-    return;
-  }
-
   // ================================================================ consumers
-  const int cw = warp;  // consumer warp 0 .. CW-1
-  const int wr = cw / WC;
-  const int wc = cw % WC;
-  const int cg = lane & 7;
-  const int rl = lane >> 3;
-  const int i0 = wr * Shape::kWarpRows + rl * R;  // first state row of this thread
-  const int c0 = wc * 64 + cg * kColsPerThread;   // first tile column of this thread
-  const bool bit4 = (lane >> 4) & 1;
-  const bool bit3 = (lane >> 3) & 1;
-  const bool writes_out = (wr == 0) && (rl == 0);  // one thread per 8 columns
-  const float scale = p.scale;
+  // lane = rl * CL + cg: row lane rl owns rows [R rl, R rl + R); column lane cg
+  // owns the 8 columns [cg * 8, cg * 8 + 8) of this warp's band.
+  const int rl = lane / CL;
+  const int cg = lane % CL;
+  const int i0 = rl * R;
+  const int cband = warp * WCOLS;  // first tile column of this warp
+  const int c0 = cband + cg * 8;   // first tile column of this thread
+  // After the reduce-scatter, lane (b4, sub, cg) with sub = rl mod (RL / 2)
+  // holds vector (b4 ? p : kv_mem) at band columns cg * 8 + sub * NV + [0, NV).
+  const bool b4 = (lane >> 4) & 1;
+  const int cred = cg * 8 + NV * (rl & (RL / 2 - 1));
 
   for (int it = 0; it < n_mine; ++it) {
     const int tile = blockIdx.x + it * gridDim.x;
     const int slice = tile % n_slices;
     const int h = (tile / n_slices) % p.H_v;
     const int b = tile / (n_slices * p.H_v);
-    const int col0 = slice * VS;
     const int stage = it % n_stages;
     const uint32_t phase = (it / n_stages) & 1;
     uint8_t* st = smem + stage * lay.bytes;
 
-    // The barrier also orders this tile's first write of the partial-sum
-    // buffers after every consumer's last read of them in the previous tile.
     const bool ok_self = mbar_wait_bounded(full0 + 8 * stage, phase);
-    const bool ok = named_bar_and(kConsumerBar, NC, ok_self);
+    const bool ok = __all_sync(0xffffffffu, ok_self);
     if (!ok_self) flag_error(kErrConsumerWait);
     const int* meta = reinterpret_cast<const int*>(st + lay.meta);
-    int L = ok ? meta[0] : 0;
+    int L = ok ? meta[0] : 0;  // one load for the whole warp: every lane sees one value
     L = L < 0 ? 0 : (L > T ? T : L);
+    if constexpr (ONE) L = L > 1 ? 1 : L;
     const int s = meta[1];
+    if (s < 0 || s >= p.pool_size) L = 0;
 
-    uint16_t* out_bh = p.out + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + col0;
-    for (int e = tid; e < (T - L) * (VS / 8); e += NC) {
-      const int t = L + e / (VS / 8);
-      const int v8 = e % (VS / 8);
-      *reinterpret_cast<uint4*>(out_bh + static_cast<size_t>(t) * p.D_v + v8 * 8) =
+    // out[b, h, :, slice * VS + cband : + WCOLS]; padded tokens get +0.0.
+    uint16_t* out_band =
+        p.out + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + slice * VS + cband;
+    for (int e = lane; e < (T - L) * (WCOLS / 8); e += 32) {
+      const int t = L + e / (WCOLS / 8);
+      const int v8 = e % (WCOLS / 8);
+      *reinterpret_cast<uint4*>(out_band + static_cast<size_t>(t) * p.D_v + v8 * 8) =
           make_uint4(0u, 0u, 0u, 0u);
     }
 
-    // S2[r][c] holds columns 2c and 2c+1 of row r as a packed fp32 pair.
-    unsigned long long S2[R][kColsPerThread / 2];
+    // Multi-token calls keep the state in fp32 registers across tokens:
+    // S2[r][c] holds columns c0 + 2c, c0 + 2c + 1 of row i0 + r as a packed
+    // pair. A single-token call keeps no state in registers: it reads its rows
+    // from the stage once for the column sums and once more for the update,
+    // and streams each new row to the pool straight from the update.
+    unsigned long long S2[ONE ? 1 : R][4];
+    const uint16_t* tile_s = reinterpret_cast<const uint16_t*>(st);
+    uint16_t* dst = p.state_pool + ((static_cast<size_t>(s) * p.H_v + h) * DK + i0) * p.D_v +
+                    slice * VS + c0;
     if (L > 0) {
-      const uint16_t* tile_s = reinterpret_cast<const uint16_t*>(st);
+      if constexpr (!ONE) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float f[8];
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0), f);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) S2[r][c] = pk(f[2 * c], f[2 * c + 1]);
+        for (int r = 0; r < R; ++r) {
+          const uint4 w = *reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0);
+          S2[r][0] = pk(bf16_lo(w.x), bf16_hi(w.x));
+          S2[r][1] = pk(bf16_lo(w.y), bf16_hi(w.y));
+          S2[r][2] = pk(bf16_lo(w.z), bf16_hi(w.z));
+          S2[r][3] = pk(bf16_lo(w.w), bf16_hi(w.w));
+        }
       }
-      const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);
+      const float4* srv = reinterpret_cast<const float4*>(st + lay.rv);  // single-token
+      const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);  // multi-token
       const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
-      const float* sd = reinterpret_cast<const float*>(st + lay.sd);
+      const float* sd = reinterpret_cast<const float*>(st + lay.gk);
       const float* sbeta = reinterpret_cast<const float*>(st + lay.beta);
       const float* skq = reinterpret_cast<const float*>(st + lay.kq);
       const uint16_t* sv = reinterpret_cast<const uint16_t*>(st + lay.v);
 
       for (int t = 0; t < L; ++t) {
-        float* buf = red + (t & 1) * (CW * 128);
-        float kr[R], qr[R], dr[R];
-#pragma unroll
-        for (int r4 = 0; r4 < R; r4 += 4) {
-          const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * DK + i0 + r4);
-          const uint2 qw = *reinterpret_cast<const uint2*>(sq + t * DK + i0 + r4);
-          const float4 dw = *reinterpret_cast<const float4*>(sd + t * DK + i0 + r4);
-          kr[r4 + 0] = bf16_lo(kw.x); kr[r4 + 1] = bf16_hi(kw.x);
-          kr[r4 + 2] = bf16_lo(kw.y); kr[r4 + 3] = bf16_hi(kw.y);
-          qr[r4 + 0] = bf16_lo(qw.x); qr[r4 + 1] = bf16_hi(qw.x);
-          qr[r4 + 2] = bf16_lo(qw.y); qr[r4 + 3] = bf16_hi(qw.y);
-          dr[r4 + 0] = dw.x; dr[r4 + 1] = dw.y; dr[r4 + 2] = dw.z; dr[r4 + 3] = dw.w;
-        }
+        // kv_mem = S_dec^T k = S^T (d k) and p = S^T (d q_s): the decay of
+        // step 1 is folded into the row vectors.
         unsigned long long m2[4], p2[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) m2[c] = p2[c] = 0ull;  // (+0.0f, +0.0f)
+        // (single-token rows are re-read from shared memory, so their loop
+        // need not be unrolled: unrolling it fully only raises register use)
+        if constexpr (ONE) {
+#pragma unroll 2
+          for (int r = 0; r < R; ++r) {
+            const float2 rv0 = reinterpret_cast<const float2*>(srv + t * DK + i0 + r)[0];
+            const unsigned long long dk2 = pk(rv0.x, rv0.x);  // {d k, d k}
+            const unsigned long long dq2 = pk(rv0.y, rv0.y);  // {d q_s, d q_s}
+            const uint4 w = *reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0);
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const unsigned long long d2 = pk(dr[r], dr[r]);
-          const unsigned long long k2 = pk(kr[r], kr[r]);
-          const unsigned long long q2 = pk(qr[r], qr[r]);
+            for (int c = 0; c < 4; ++c) {
+              const unsigned long long sr = pk(bf16_lo(wv[c]), bf16_hi(wv[c]));
+              m2[c] = fma2(sr, dk2, m2[c]);  // steps 1-2: kv_mem partial
+              p2[c] = fma2(sr, dq2, p2[c]);  // S_dec^T q_s partial
+            }
+          }
+        } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            S2[r][c] = mul2(S2[r][c], d2);      // step 1: decay row r
-            m2[c] = fma2(S2[r][c], k2, m2[c]);  // step 2: kv_mem partial
-            p2[c] = fma2(S2[r][c], q2, p2[c]);  // S^T q partial (scale applied later)
+          for (int r4 = 0; r4 < R; r4 += 4) {
+            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * DK + i0 + r4);
+            const uint2 qw = *reinterpret_cast<const uint2*>(sq + t * DK + i0 + r4);
+            const float4 dw = *reinterpret_cast<const float4*>(sd + t * DK + i0 + r4);
+            const float kr[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
+            const float qr[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
+            const float dr[4] = {dw.x, dw.y, dw.z, dw.w};
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              const float dk = dr[rr] * kr[rr], dq = dr[rr] * qr[rr];
+              const unsigned long long dk2 = pk(dk, dk);
+              const unsigned long long dq2 = pk(dq, dq);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                m2[c] = fma2(S2[r4 + rr][c], dk2, m2[c]);  // steps 1-2: kv_mem partial
+                p2[c] = fma2(S2[r4 + rr][c], dq2, p2[c]);  // S_dec^T q partial (unscaled)
+              }
+            }
           }
         }
-        float m[kColsPerThread], pp[kColsPerThread];
+        // Reduce-scatter over the row lanes: xor 16 splits (kv_mem | p), then
+        // xor 8 (and 4 for 8 row lanes, and 2 for 16) halve the columns.
+        float x[8];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float2 mv = upk(m2[c]);
           const float2 pv = upk(p2[c]);
-          m[2 * c] = mv.x; m[2 * c + 1] = mv.y;
-          pp[2 * c] = pv.x; pp[2 * c + 1] = pv.y;
-        }
-        // Reduce-scatter over the 4 row lanes: xor 16 splits (kv_mem | p), xor 8
-        // splits the 8 columns into halves. Lane (bit4, bit3, cg) ends with the
-        // warp sum of vector (bit4 ? p : kv_mem) at columns cg*8 + bit3*4 + 0..3.
-        float x[kColsPerThread];
-#pragma unroll
-        for (int c = 0; c < kColsPerThread; ++c) {
-          const float send = bit4 ? m[c] : pp[c];
-          const float keep = bit4 ? pp[c] : m[c];
-          x[c] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+          const float s0 = b4 ? mv.x : pv.x, s1 = b4 ? mv.y : pv.y;
+          const float k0 = b4 ? pv.x : mv.x, k1 = b4 ? pv.y : mv.y;
+          x[2 * c] = k0 + __shfl_xor_sync(0xffffffffu, s0, 16);
+          x[2 * c + 1] = k1 + __shfl_xor_sync(0xffffffffu, s1, 16);
         }
         float y[4];
+        {
+          const bool bit = (lane >> 3) & 1;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float send = bit3 ? x[c] : x[c + 4];
-          const float keep = bit3 ? x[c + 4] : x[c];
-          y[c] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-        *reinterpret_cast<float4*>(buf + (cw * 32 + lane) * 4) = make_float4(y[0], y[1], y[2], y[3]);
-        named_bar_sync(kConsumerBar, NC);
-        // kv_mem of this thread's 8 columns: the sum over the warp rows of the
-        // partials held by lanes (0, 0, cg) and (0, 1, cg) of each warp.
-        float mem[kColsPerThread];
-#pragma unroll
-        for (int c = 0; c < kColsPerThread; ++c) mem[c] = 0.0f;
-#pragma unroll
-        for (int w = 0; w < WR; ++w) {
-          const float* src = buf + ((w * WC + wc) * 32 + cg) * 4;
-          const float4 lo = *reinterpret_cast<const float4*>(src);
-          const float4 hi = *reinterpret_cast<const float4*>(src + 8 * 4);
-          mem[0] += lo.x; mem[1] += lo.y; mem[2] += lo.z; mem[3] += lo.w;
-          mem[4] += hi.x; mem[5] += hi.y; mem[6] += hi.z; mem[7] += hi.w;
-        }
-        float vv[kColsPerThread];
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(sv + t * VS + c0), vv);
-        const float bt = sbeta[t];
-        float dl[kColsPerThread];
-#pragma unroll
-        for (int c = 0; c < kColsPerThread; ++c) dl[c] = (vv[c] - mem[c]) * bt;  // step 3
-        if (writes_out) {
-          float pj[kColsPerThread];
-#pragma unroll
-          for (int c = 0; c < kColsPerThread; ++c) pj[c] = 0.0f;
-#pragma unroll
-          for (int w = 0; w < WR; ++w) {
-            const float* src = buf + ((w * WC + wc) * 32 + 16 + cg) * 4;
-            const float4 lo = *reinterpret_cast<const float4*>(src);
-            const float4 hi = *reinterpret_cast<const float4*>(src + 8 * 4);
-            pj[0] += lo.x; pj[1] += lo.y; pj[2] += lo.z; pj[3] += lo.w;
-            pj[4] += hi.x; pj[5] += hi.y; pj[6] += hi.z; pj[7] += hi.w;
+          for (int c = 0; c < 4; ++c) {
+            const float send = bit ? x[c] : x[c + 4];
+            const float keep = bit ? x[c + 4] : x[c];
+            y[c] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
           }
-          const float kq = skq[t];
-          float o[kColsPerThread];
-#pragma unroll
-          for (int c = 0; c < kColsPerThread; ++c) o[c] = fmaf(dl[c], kq, pj[c] * scale);  // step 4
-          uint4 ow;
-          ow.x = pack_bf16x2(o[0], o[1]);
-          ow.y = pack_bf16x2(o[2], o[3]);
-          ow.z = pack_bf16x2(o[4], o[5]);
-          ow.w = pack_bf16x2(o[6], o[7]);
-          *reinterpret_cast<uint4*>(out_bh + static_cast<size_t>(t) * p.D_v + c0) = ow;
         }
+        float red[NV];
+        if constexpr (NV == 4) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) red[c] = y[c];
+        } else {
+          float z[2];
+          const bool bit = (lane >> 2) & 1;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float send = bit ? y[c] : y[c + 2];
+            const float keep = bit ? y[c + 2] : y[c];
+            z[c] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+          }
+          if constexpr (NV == 2) {
+            red[0] = z[0];
+            red[1] = z[1];
+          } else {
+            const bool bit1 = (lane >> 1) & 1;
+            const float send = bit1 ? z[0] : z[1];
+            const float keep = bit1 ? z[1] : z[0];
+            red[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+          }
+        }
+        // kv_mem lanes: delta = (v - kv_mem) * beta (step 3), then handed to the
+        // p lane of the same columns, which writes o (step 4).
+        float dlt[NV];
+        {
+          const float bt = sbeta[t];
+          if constexpr (NV == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(sv + t * VS + cband + cred);
+            dlt[0] = (bf16_lo(w.x) - red[0]) * bt;
+            dlt[1] = (bf16_hi(w.x) - red[1]) * bt;
+            dlt[2] = (bf16_lo(w.y) - red[2]) * bt;
+            dlt[3] = (bf16_hi(w.y) - red[3]) * bt;
+          } else if constexpr (NV == 2) {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(sv + t * VS + cband + cred);
+            dlt[0] = (bf16_lo(w) - red[0]) * bt;
+            dlt[1] = (bf16_hi(w) - red[1]) * bt;
+          } else {
+            dlt[0] = (bf16_bits_to_f32(sv[t * VS + cband + cred]) - red[0]) * bt;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < NV; ++c) {
+          const float other = __shfl_xor_sync(0xffffffffu, dlt[c], 16);
+          if (b4) dlt[c] = other;
+        }
+        if (b4) {
+          const float kq = skq[t];
+          // single-token p already carries the query scale; multi-token p does not
+          const float ps = ONE ? 1.0f : p.scale;
+          uint16_t* dst = out_band + static_cast<size_t>(t) * p.D_v + cred;
+          if constexpr (NV == 4) {
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(pack_bf16x2(fmaf(dlt[0], kq, red[0] * ps), fmaf(dlt[1], kq, red[1] * ps)),
+                           pack_bf16x2(fmaf(dlt[2], kq, red[2] * ps), fmaf(dlt[3], kq, red[3] * ps)));  // step 4
+          } else if constexpr (NV == 2) {
+            *reinterpret_cast<uint32_t*>(dst) =
+                pack_bf16x2(fmaf(dlt[0], kq, red[0] * ps), fmaf(dlt[1], kq, red[1] * ps));  // step 4
+          } else {
+            *dst = f32_to_bf16_bits(fmaf(dlt[0], kq, red[0] * ps));  // step 4
+          }
+        }
+        // every lane gathers delta of its own 8 columns from the kv_mem lanes
+        // (b4 = 0, sub = sb, cg) = lane sb * CL + cg
+        float dl[8];
+#pragma unroll
+        for (int sb = 0; sb < RL / 2; ++sb)
+#pragma unroll
+          for (int c = 0; c < NV; ++c)
+            dl[sb * NV + c] = __shfl_sync(0xffffffffu, dlt[c], sb * CL + cg);
         unsigned long long dl2[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) dl2[c] = pk(dl[2 * c], dl[2 * c + 1]);
+        // steps 1 and 3: S_new = d S + k delta^T
+        if constexpr (ONE) {
+#pragma unroll 2
+          for (int r = 0; r < R; ++r) {
+            const float2 rv1 = reinterpret_cast<const float2*>(srv + t * DK + i0 + r)[1];
+            const unsigned long long d2 = pk(rv1.x, rv1.x);  // {d, d}
+            const unsigned long long k2 = pk(rv1.y, rv1.y);  // {k, k}
+            const uint4 w = *reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0);
+            const float2 n0 = upk(fma2(pk(bf16_lo(w.x), bf16_hi(w.x)), d2, mul2(k2, dl2[0])));
+            const float2 n1 = upk(fma2(pk(bf16_lo(w.y), bf16_hi(w.y)), d2, mul2(k2, dl2[1])));
+            const float2 n2 = upk(fma2(pk(bf16_lo(w.z), bf16_hi(w.z)), d2, mul2(k2, dl2[2])));
+            const float2 n3 = upk(fma2(pk(bf16_lo(w.w), bf16_hi(w.w)), d2, mul2(k2, dl2[3])));
+            // bf16 round-to-nearest-even, once per call, straight to the slot
+            __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * p.D_v),
+                   make_uint4(pack_bf16x2(n0.x, n0.y), pack_bf16x2(n1.x, n1.y),
+                              pack_bf16x2(n2.x, n2.y), pack_bf16x2(n3.x, n3.y)));
+          }
+        } else {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const unsigned long long k2 = pk(kr[r], kr[r]);
+          for (int r4 = 0; r4 < R; r4 += 4) {
+            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * DK + i0 + r4);
+            const float4 dw = *reinterpret_cast<const float4*>(sd + t * DK + i0 + r4);
+            const float kr[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
+            const float dr[4] = {dw.x, dw.y, dw.z, dw.w};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) S2[r][c] = fma2(k2, dl2[c], S2[r][c]);  // step 3: S += k delta^T
+            for (int rr = 0; rr < 4; ++rr) {
+              const unsigned long long d2 = pk(dr[rr], dr[rr]);
+              const unsigned long long k2 = pk(kr[rr], kr[rr]);
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                S2[r4 + rr][c] = fma2(S2[r4 + rr][c], d2, mul2(k2, dl2[c]));
+            }
+          }
         }
       }
     }
-    // This warp is done reading the input stage: the producer may refill it.
+    // This warp has read everything it needs from the stage: give it back.
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * stage);
 
-    // Write the new tile into the next output buffer once its last store has
-    // read it, then hand it to the storer.
-    const int ob = it % kOutBuffers;
-    const uint32_t ophase = (it / kOutBuffers) & 1;
-    bool ok_out = true;
-    if (L > 0) {
-      ok_out = mbar_wait_bounded(oempty0 + 8 * ob, ophase ^ 1);
-      if (!ok_out) flag_error(kErrConsumerWait);
-      uint16_t* out_tile = reinterpret_cast<uint16_t*>(obuf + ob * Shape::kStateBytes);
-      // bf16, round-to-nearest-even, once per call
+    if (!ONE && L > 0) {
+      // The new state, bf16 round-to-nearest-even once per call, streamed from
+      // registers to the slot with 16-byte stores.
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         uint4 o;
-        float2 v;
-        v = upk(S2[r][0]); o.x = pack_bf16x2(v.x, v.y);
-        v = upk(S2[r][1]); o.y = pack_bf16x2(v.x, v.y);
-        v = upk(S2[r][2]); o.z = pack_bf16x2(v.x, v.y);
-        v = upk(S2[r][3]); o.w = pack_bf16x2(v.x, v.y);
-        *reinterpret_cast<uint4*>(out_tile + (i0 + r) * VS + c0) = o;
+        {
+          float2 v;
+          v = upk(S2[r][0]); o.x = pack_bf16x2(v.x, v.y);
+          v = upk(S2[r][1]); o.y = pack_bf16x2(v.x, v.y);
+          v = upk(S2[r][2]); o.z = pack_bf16x2(v.x, v.y);
+          v = upk(S2[r][3]); o.w = pack_bf16x2(v.x, v.y);
+        }
+        __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * p.D_v), o);
       }
-      fence_proxy_async_smem();
-    } else {
-      // Nothing is written; still wait for the buffer so the (length, slot)
-      // words below are not changed under a store that is reading them.
-      ok_out = mbar_wait_bounded(oempty0 + 8 * ob, ophase ^ 1);
-      if (!ok_out) flag_error(kErrConsumerWait);
     }
-    if (tid == 0) {
-      ometa[4 * ob + 0] = L;
-      ometa[4 * ob + 1] = s;
-      ometa[4 * ob + 2] = (ok && ok_out) ? 0 : 1;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(ofull0 + 8 * ob);
   }
 }
 
