@@ -177,20 +177,21 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
 
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  // The pool seen as a 3-D bf16 array: [pool * H_v * D_k rows][D_v / C blocks][C
-  // columns] with C = min(VS, 256), so one box {C, VS / C, D_k} is a whole tile
-  // and, for VS = D_v, one contiguous (slot, head) state.
+  // The pool seen as a 3-D bf16 array [D_v / 64 column blocks][pool * H_v * D_k
+  // rows][64 columns] (row stride D_v * 2 bytes, block stride 128 bytes). One
+  // box {64, D_k, VS / 64} is a whole tile and lands in shared memory as
+  // [block][row][64 columns] with the 128-byte swizzle: within each 128-byte
+  // row segment, 16-byte chunk c is stored at position c ^ (row % 8), so the
+  // consumers' 16-byte reads of different rows fall in different banks.
   CUtensorMap map;
-  constexpr int C = Shape::kBoxCols;
-  const cuuint64_t gdim[3] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(p.D_v / C),
-                              static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK};
-  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(C) * 2,
-                                 static_cast<cuuint64_t>(p.D_v) * 2};
-  const cuuint32_t box[3] = {C, Shape::kBoxParts, DK};
+  const cuuint64_t gdim[3] = {64, static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK,
+                              static_cast<cuuint64_t>(p.D_v / 64)};
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(p.D_v) * 2, 128};
+  const cuuint32_t box[3] = {64, DK, VS / 64};
   const cuuint32_t estride[3] = {1, 1, 1};
   const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                              const_cast<uint16_t*>(p.state_pool), gdim, gstride, box, estride,
-                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled failed");

@@ -78,14 +78,44 @@ struct TmaShape {
   static constexpr int kConsumers = kConsumerWarps * 32;
   static constexpr int kThreads = kConsumers + 32;  // + the producer warp
   static constexpr int kStateBytes = DK * VS * 2;
-  static constexpr int kBoxCols = VS < 256 ? VS : 256;  // TMA box extents: columns,
-  static constexpr int kBoxParts = VS / kBoxCols;       // column blocks, rows (= D_k)
+  // Per-token stride of the per-row arrays: each row lane's R entries are
+  // padded to R + 4, so the row lanes of one quarter-warp read different banks.
+  static constexpr int kTokStride = DK + 4 * kRowLanes;
   static_assert(DK == 64 || DK == 128, "D_k must be 64 or 128");
   static_assert(R == 8 || R == 16, "8 or 16 rows per thread");
   static_assert(kRowLanes >= 4 && kRowLanes <= 16, "4 to 16 row lanes");
   static_assert(VS % kWarpCols == 0 && kConsumerWarps >= 1 && kConsumerWarps <= 16,
                 "one to sixteen consumer warps per tile");
 };
+
+// Row ownership. Row lane rl owns rows r * RL + row_perm(rl), r < R: the rows
+// that one quarter-warp reads together then differ in bit 2 (8 row lanes) or
+// in bits 1-2 (16 row lanes) of the row index, so with the 128-byte swizzle of
+// the state tile their 16-byte reads fall in different banks.
+template <int RL>
+__host__ __device__ constexpr int row_perm(int rl) {
+  return RL == 8 ? ((rl >> 1) | ((rl & 1) << 2))
+                 : (RL == 16 ? (2 * (rl & 3) + ((rl >> 2) & 1) + 8 * (rl >> 3)) : rl);
+}
+
+// Where row i sits in "owner order": the R rows of row lane rl are stored
+// contiguously at [rl * (R + 4), rl * (R + 4) + R), so per-row vectors load as
+// vectors and the four padding entries stagger the row lanes across banks.
+template <int RL, int R>
+__host__ __device__ constexpr int owner_slot(int i) {
+  const int x = i % RL;
+  const int r = i / RL;
+  const int rl = RL == 8 ? (((x & 3) << 1) | (x >> 2))
+                         : (RL == 16 ? (4 * (((x >> 3) << 1) | (x & 1)) + ((x >> 1) & 3)) : x);
+  return rl * (R + 4) + r;
+}
+
+// Byte offset of (row i, 16-byte chunk holding column col) in a state tile
+// loaded with the 128-byte swizzle as [col / 64][row][64 columns].
+template <int DK>
+__device__ __forceinline__ int swz_offset(int i, int col) {
+  return ((((col >> 6) * DK + i)) << 7) + ((((col >> 3) & 7) ^ (i & 7)) << 4);
+}
 
 // Byte offsets inside one stage, for T padded tokens.
 struct StageLayout {
@@ -98,11 +128,14 @@ template <int DK, int VS, int R, bool ONE>
 __host__ __device__ inline StageLayout stage_layout(int T) {
   StageLayout s;
   s.v = TmaShape<DK, VS, R>::kStateBytes;  // bf16 [T][VS]   value rows of the slice
-  s.k = s.v + T * VS * 2;               // bf16 [T][DK]   key rows
-  s.q = s.k + T * DK * 2;               // bf16 [T][DK]   query rows
-  s.gk = s.q + T * DK * 2;              // fp32 [T][DK]   gk rows (multi-token: then d = exp(g + gk))
-  s.rv = s.gk + T * DK * 4;             // fp32x4 [T][DK] {d*k, d*q*scale, d, k} (single-token only)
-  s.raw = s.rv + (ONE ? T * DK * 16 : 0);  // u32 [2][8]  gate scalar words
+  // per-row arrays: [T][TS] with TS = DK + 4 * row lanes; rows arrive in natural
+  // order and the producer rewrites them in owner order (see owner_slot)
+  constexpr int TS = TmaShape<DK, VS, R>::kTokStride;
+  s.k = s.v + T * VS * 2;               // bf16 [T][TS]   key rows
+  s.q = s.k + T * TS * 2;               // bf16 [T][TS]   query rows
+  s.gk = s.q + T * TS * 2;              // fp32 [T][TS]   gk rows (multi-token: then d = exp(g + gk))
+  s.rv = s.gk + T * TS * 4;             // fp32x4 [T][TS] {d*k, d*q*scale, d, k} (single-token only)
+  s.raw = s.rv + (ONE ? T * TS * 16 : 0);  // u32 [2][8]  gate scalar words
   s.beta = s.raw + 64;                  // fp32 [8]
   s.kq = s.beta + 32;                   // fp32 [8]       k . (q * scale)
   s.meta = s.kq + 32;                   // int32 [4]      length, slot
@@ -254,6 +287,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
   constexpr int CL = Shape::kColLanes;
   constexpr int WCOLS = Shape::kWarpCols;
   constexpr int NV = 16 / RL;  // reduced values per lane after the reduce-scatter: 4, 2 or 1
+  constexpr int TS = Shape::kTokStride;
   const int T = p.T;
   const StageLayout lay = stage_layout<DK, VS, RR, ONE>(T);
 
@@ -331,13 +365,15 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
           meta[1] = s;
           if (L > 0) {
             mbar_expect_tx(rawb, Shape::kStateBytes + L * (VS * 2 + DK * 8));
-            tma_load_3d(smem_addr(st), &pool_map, 0, col0 / Shape::kBoxCols,
-                        (s * p.H_v + h) * DK, rawb);
+            tma_load_3d(smem_addr(st), &pool_map, 0, (s * p.H_v + h) * DK, col0 / 64, rawb);
             const size_t qk_off = (static_cast<size_t>(b) * p.H_qk + hq) * T * DK;
             const size_t gk_off = (static_cast<size_t>(b) * p.H_v + h) * T * DK;
-            bulk_load(smem_addr(st + lay.k), p.key + qk_off, L * DK * 2, rawb);
-            bulk_load(smem_addr(st + lay.q), p.query + qk_off, L * DK * 2, rawb);
-            bulk_load(smem_addr(st + lay.gk), p.gk + gk_off, L * DK * 4, rawb);
+            for (int t = 0; t < L; ++t) {  // one row of each per token (padded stride)
+              bulk_load(smem_addr(st + lay.k + t * TS * 2), p.key + qk_off + t * DK, DK * 2, rawb);
+              bulk_load(smem_addr(st + lay.q + t * TS * 2), p.query + qk_off + t * DK, DK * 2,
+                        rawb);
+              bulk_load(smem_addr(st + lay.gk + t * TS * 4), p.gk + gk_off + t * DK, DK * 4, rawb);
+            }
             const uint16_t* vsrc =
                 p.value + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + col0;
             for (int t = 0; t < L; ++t)
@@ -385,6 +421,8 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         float4* srv = reinterpret_cast<float4*>(st + lay.rv);
         const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);
         const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
+        uint16_t* skw = reinterpret_cast<uint16_t*>(st + lay.k);
+        uint16_t* sqw = reinterpret_cast<uint16_t*>(st + lay.q);
         float dtb = 0.0f, dsc = 0.0f;
         if constexpr (GATED) {
           if (L > 0) {
@@ -407,19 +445,33 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
             gt = __uint_as_float(rawv[t]);
             bt = bf16_in_word(rawv[8 + t], p.beta + gi);
           }
+          // Row vectors go to owner order (see owner_slot): read every row of
+          // this token first, then write, so the in-place permutation of the
+          // multi-token arrays is safe.
           float kq = 0.0f;
+          float dv[E], kv[E], qv[E];
+          uint16_t kb[E], qb[E];
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const int i = lane + 32 * e;
-            const float d = expf(gt + sgk[t * DK + i]);  // exp(g) * exp(gk) as one exponential
-            const float kv = bf16_bits_to_f32(sk[t * DK + i]);
-            const float qs = bf16_bits_to_f32(sq[t * DK + i]) * p.scale;
+            dv[e] = expf(gt + sgk[t * TS + i]);  // exp(g) * exp(gk) as one exponential
+            kb[e] = sk[t * TS + i];
+            qb[e] = sq[t * TS + i];
+            kv[e] = bf16_bits_to_f32(kb[e]);
+            qv[e] = bf16_bits_to_f32(qb[e]) * p.scale;
+            kq = fmaf(kv[e], qv[e], kq);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const int o = t * TS + owner_slot<RL, R>(lane + 32 * e);
             if constexpr (ONE) {
-              srv[t * DK + i] = make_float4(d * kv, d * qs, d, kv);
+              srv[o] = make_float4(dv[e] * kv[e], dv[e] * qv[e], dv[e], kv[e]);
             } else {
-              sgk[t * DK + i] = d;
+              sgk[o] = dv[e];
+              skw[o] = kb[e];
+              sqw[o] = qb[e];
             }
-            kq = fmaf(kv, qs, kq);
           }
           kq = warp_sum(kq);
           __syncwarp();
@@ -444,11 +496,13 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
   }
 
   // ================================================================ consumers
-  // lane = rl * CL + cg: row lane rl owns rows [R rl, R rl + R); column lane cg
-  // owns the 8 columns [cg * 8, cg * 8 + 8) of this warp's band.
+  // lane = rl * CL + cg: row lane rl owns rows r * RL + row_perm(rl), r < R
+  // (their per-row vectors sit at owner slots [rl * R, rl * R + R)); column
+  // lane cg owns the 8 columns [cg * 8, cg * 8 + 8) of this warp's band.
   const int rl = lane / CL;
   const int cg = lane % CL;
-  const int i0 = rl * R;
+  const int i0 = rl * (R + 4);      // first owner slot of this thread
+  const int rp = row_perm<RL>(rl);  // row of slot i0 + r is r * RL + rp
   const int cband = warp * WCOLS;  // first tile column of this warp
   const int c0 = cband + cg * 8;   // first tile column of this thread
   // After the reduce-scatter, lane (b4, sub, cg) with sub = rl mod (RL / 2)
@@ -491,14 +545,13 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     // from the stage once for the column sums and once more for the update,
     // and streams each new row to the pool straight from the update.
     unsigned long long S2[ONE ? 1 : R][4];
-    const uint16_t* tile_s = reinterpret_cast<const uint16_t*>(st);
-    uint16_t* dst = p.state_pool + ((static_cast<size_t>(s) * p.H_v + h) * DK + i0) * p.D_v +
-                    slice * VS + c0;
+    uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
+                    slice * VS + c0;  // + row * D_v
     if (L > 0) {
       if constexpr (!ONE) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const uint4 w = *reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0);
+          const uint4 w = *reinterpret_cast<const uint4*>(st + swz_offset<DK>(r * RL + rp, c0));
           S2[r][0] = pk(bf16_lo(w.x), bf16_hi(w.x));
           S2[r][1] = pk(bf16_lo(w.y), bf16_hi(w.y));
           S2[r][2] = pk(bf16_lo(w.z), bf16_hi(w.z));
@@ -524,10 +577,10 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         if constexpr (ONE) {
 #pragma unroll 2
           for (int r = 0; r < R; ++r) {
-            const float2 rv0 = reinterpret_cast<const float2*>(srv + t * DK + i0 + r)[0];
+            const float2 rv0 = reinterpret_cast<const float2*>(srv + t * TS + i0 + r)[0];
             const unsigned long long dk2 = pk(rv0.x, rv0.x);  // {d k, d k}
             const unsigned long long dq2 = pk(rv0.y, rv0.y);  // {d q_s, d q_s}
-            const uint4 w = *reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0);
+            const uint4 w = *reinterpret_cast<const uint4*>(st + swz_offset<DK>(r * RL + rp, c0));
             const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -539,9 +592,9 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         } else {
 #pragma unroll
           for (int r4 = 0; r4 < R; r4 += 4) {
-            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * DK + i0 + r4);
-            const uint2 qw = *reinterpret_cast<const uint2*>(sq + t * DK + i0 + r4);
-            const float4 dw = *reinterpret_cast<const float4*>(sd + t * DK + i0 + r4);
+            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * TS + i0 + r4);
+            const uint2 qw = *reinterpret_cast<const uint2*>(sq + t * TS + i0 + r4);
+            const float4 dw = *reinterpret_cast<const float4*>(sd + t * TS + i0 + r4);
             const float kr[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
             const float qr[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
             const float dr[4] = {dw.x, dw.y, dw.z, dw.w};
@@ -658,24 +711,24 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         if constexpr (ONE) {
 #pragma unroll 2
           for (int r = 0; r < R; ++r) {
-            const float2 rv1 = reinterpret_cast<const float2*>(srv + t * DK + i0 + r)[1];
+            const float2 rv1 = reinterpret_cast<const float2*>(srv + t * TS + i0 + r)[1];
             const unsigned long long d2 = pk(rv1.x, rv1.x);  // {d, d}
             const unsigned long long k2 = pk(rv1.y, rv1.y);  // {k, k}
-            const uint4 w = *reinterpret_cast<const uint4*>(tile_s + (i0 + r) * VS + c0);
+            const uint4 w = *reinterpret_cast<const uint4*>(st + swz_offset<DK>(r * RL + rp, c0));
             const float2 n0 = upk(fma2(pk(bf16_lo(w.x), bf16_hi(w.x)), d2, mul2(k2, dl2[0])));
             const float2 n1 = upk(fma2(pk(bf16_lo(w.y), bf16_hi(w.y)), d2, mul2(k2, dl2[1])));
             const float2 n2 = upk(fma2(pk(bf16_lo(w.z), bf16_hi(w.z)), d2, mul2(k2, dl2[2])));
             const float2 n3 = upk(fma2(pk(bf16_lo(w.w), bf16_hi(w.w)), d2, mul2(k2, dl2[3])));
             // bf16 round-to-nearest-even, once per call, straight to the slot
-            __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * p.D_v),
+            __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r * RL + rp) * p.D_v),
                    make_uint4(pack_bf16x2(n0.x, n0.y), pack_bf16x2(n1.x, n1.y),
                               pack_bf16x2(n2.x, n2.y), pack_bf16x2(n3.x, n3.y)));
           }
         } else {
 #pragma unroll
           for (int r4 = 0; r4 < R; r4 += 4) {
-            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * DK + i0 + r4);
-            const float4 dw = *reinterpret_cast<const float4*>(sd + t * DK + i0 + r4);
+            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * TS + i0 + r4);
+            const float4 dw = *reinterpret_cast<const float4*>(sd + t * TS + i0 + r4);
             const float kr[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
             const float dr[4] = {dw.x, dw.y, dw.z, dw.w};
 #pragma unroll
@@ -707,7 +760,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
           v = upk(S2[r][2]); o.z = pack_bf16x2(v.x, v.y);
           v = upk(S2[r][3]); o.w = pack_bf16x2(v.x, v.y);
         }
-        __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * p.D_v), o);
+        __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r * RL + rp) * p.D_v), o);
       }
     }
   }
