@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from gated_delta_rule_recurrent_b200 import metrics, workloads  # noqa: E402
+from gated_delta_rule_recurrent_b200 import distributed, metrics, workloads  # noqa: E402
 
 METRIC = "decode tokens/s and achieved HBM GB/s vs ~8 TB/s peak for gated-delta step"
 NOMINAL_HBM_GBS = 8000.0
@@ -48,13 +48,6 @@ TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gated_B512_H64_64x512_dr
 
 
 # --------------------------------------------------------------------------- helpers
-
-def _dist_env():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
-
 
 def measured_hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -206,12 +199,78 @@ def oracle_tokens_per_s(x, gated, items_per_call, budget_s, items_order=None):
     return tokens / elapsed, tokens, items_done, elapsed
 
 
+def measure_e2e(args, w, x, xd, out, dev, step, barrier, max_over_ranks, world, n_tokens):
+    """End to end through the public API with host buffers.
+
+    Every timed step copies its per-token inputs from pinned host memory to the
+    device, runs the decode call, and copies its output back to pinned host
+    memory; the state pool stays resident, as it does in serving. Steps are
+    pipelined over three streams with double-buffered device inputs and
+    outputs, so step i+1's upload and step i-1's download overlap step i's
+    kernel; the state pool's updates stay in call order on the compute stream.
+    """
+    gated = w.gated
+    per_step = ["query", "key", "value", "gk", "actual_seq_lengths", "ssm_state_indices",
+                "num_accepted_tokens"] + (["a", "b"] if gated else ["beta", "g"])
+    host = {k: x[k].pin_memory() for k in per_step}
+    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(host[k].numel() * host[k].element_size() for k in per_step)
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    dev_in = [{k: torch.empty_like(xd[k]) for k in per_step} for _ in range(2)]
+    dev_out = [out, torch.empty_like(out)]
+    up, comp, down = (torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    ev_in = [torch.cuda.Event() for _ in range(2)]         # inputs of a slot uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]       # kernel done with a slot's inputs
+    ev_done = [torch.cuda.Event() for _ in range(2)]       # kernel wrote a slot's output
+    ev_fetched = [torch.cuda.Event() for _ in range(2)]    # output of a slot downloaded
+    for e in ev_used + ev_fetched:
+        e.record(torch.cuda.current_stream(dev))
+
+    def run(n):
+        for i in range(n):
+            j = i % 2
+            with torch.cuda.stream(up):
+                up.wait_event(ev_used[j])
+                for k in per_step:
+                    dev_in[j][k].copy_(host[k], non_blocking=True)
+                ev_in[j].record(up)
+            with torch.cuda.stream(comp):
+                comp.wait_event(ev_in[j])
+                comp.wait_event(ev_fetched[j])
+                step(o=dev_out[j], inputs=dev_in[j])
+                ev_used[j].record(comp)
+                ev_done[j].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_done[j])
+                host_out[j].copy_(dev_out[j], non_blocking=True)
+                ev_fetched[j].record(down)
+
+    run(max(1, args.warmup))
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(up)
+    run(args.steps)
+    down.wait_event(ev_fetched[(args.steps - 1) % 2])
+    e1.record(down)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    tokens = distributed.sum_over_ranks(n_tokens * args.steps, dev)
+    return {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": e2e_ms / args.steps,
+            "pipelining": "upload, kernel and download on 3 streams, double-buffered"}
+
+
 # --------------------------------------------------------------------------- CUDA arm
 
 def run_gdr(args):
     import torch.distributed as dist
 
-    world, rank, local = _dist_env()
+    world, rank, local = distributed.rank_env()
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
@@ -230,7 +289,7 @@ def run_gdr(args):
         w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch, pool=args.batch)
     gated = w.gated
     # Each rank decodes its own batch: independent sequences and pool slots.
-    x = workloads.make_inputs(w, seed=w.seed + 7919 * rank)
+    x = workloads.make_inputs(w, seed=distributed.rank_seed(w.seed, rank))
     xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     out = torch.empty(w.B, w.H_v, w.T, w.D_v, dtype=torch.bfloat16, device=dev)
     lengths = x["actual_seq_lengths"].tolist()
@@ -239,27 +298,24 @@ def run_gdr(args):
                                            gated)
     stream = torch.cuda.current_stream(dev)
 
-    def step(o=out):
+    def step(o=out, inputs=None):
+        z = xd if inputs is None else {**xd, **inputs}
         if gated:
-            gdr.decode_gated(xd["query"], xd["key"], xd["value"], xd["a"], xd["b"],
-                             xd["dt_bias"], xd["decay_scale"], xd["state_pool"],
-                             xd["actual_seq_lengths"], xd["ssm_state_indices"], xd["gk"],
-                             xd["num_accepted_tokens"], xd["scale_value"], out=o)
+            gdr.decode_gated(z["query"], z["key"], z["value"], z["a"], z["b"],
+                             z["dt_bias"], z["decay_scale"], z["state_pool"],
+                             z["actual_seq_lengths"], z["ssm_state_indices"], z["gk"],
+                             z["num_accepted_tokens"], z["scale_value"], out=o)
         else:
-            gdr.decode(xd["query"], xd["key"], xd["value"], xd["beta"], xd["state_pool"],
-                       xd["actual_seq_lengths"], xd["ssm_state_indices"], xd["g"], xd["gk"],
-                       xd["num_accepted_tokens"], xd["scale_value"], out=o)
+            gdr.decode(z["query"], z["key"], z["value"], z["beta"], z["state_pool"],
+                       z["actual_seq_lengths"], z["ssm_state_indices"], z["g"], z["gk"],
+                       z["num_accepted_tokens"], z["scale_value"], out=o)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return distributed.max_over_ranks(v, dev)
 
     sampler = ClockSampler(local)
     sampler.wait_first()
@@ -287,6 +343,7 @@ def run_gdr(args):
     barrier()
     launches = K  # one kernel per step (the decode kernel)
     region_ms = max_over_ranks(region0.elapsed_time(region1))
+    total_tokens = distributed.sum_over_ranks(n_tokens * K, dev)
     kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
     kernel_ms = max_over_ranks(kernel_ms)
     clocks = sampler.summary(host_t0, host_t1)
@@ -296,36 +353,8 @@ def run_gdr(args):
     # pool stays resident on the device, as it does in serving.
     e2e = None
     if not args.no_e2e:
-        per_step = ["query", "key", "value", "gk", "actual_seq_lengths", "ssm_state_indices",
-                    "num_accepted_tokens"] + (["a", "b"] if gated else ["beta", "g"])
-        host = {k: x[k].pin_memory() for k in per_step}
-        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(host[k].numel() * host[k].element_size() for k in per_step)
-        d2h = host_out.numel() * host_out.element_size()
-
-        def e2e_step():
-            for k in per_step:
-                xd[k].copy_(host[k], non_blocking=True)
-            step()
-            host_out.copy_(out, non_blocking=True)
-
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize(dev)
-        e0.record(stream)
-        for _ in range(K):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": world * n_tokens * K / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e2e_ms / K}
+        e2e = measure_e2e(args, w, x, xd, out, dev, step, barrier, max_over_ranks, world,
+                          n_tokens)
     sampler.stop()
 
     cpu = None
@@ -343,7 +372,7 @@ def run_gdr(args):
 
     peak, peak_kind = measured_hbm_peak()
     achieved = step_bytes / (kernel_ms / 1e3) / 1e9
-    value = world * n_tokens * K / (region_ms / 1e3)
+    value = total_tokens / (region_ms / 1e3)
     line = {
         "metric": METRIC,
         "value": value,
@@ -385,7 +414,7 @@ def run_gdr(args):
 # --------------------------------------------------------------------------- oracle arm
 
 def run_reference(args):
-    world, rank, _ = _dist_env()
+    world, rank, _ = distributed.rank_env()
     if rank != 0:
         return  # rank 0 alone times the CPU oracle
     w = workloads.workload(args.workload)

@@ -113,7 +113,7 @@ __host__ __device__ constexpr int owner_slot(int i) {
 // Byte offset of (row i, 16-byte chunk holding column col) in a state tile
 // loaded with the 128-byte swizzle as [col / 64][row][64 columns].
 template <int DK>
-__device__ __forceinline__ int swz_offset(int i, int col) {
+__host__ __device__ __forceinline__ int swz_offset(int i, int col) {
   return ((((col >> 6) * DK + i)) << 7) + ((((col >> 3) & 7) ^ (i & 7)) << 4);
 }
 
