@@ -16,6 +16,7 @@
 
 #include "gdr.h"
 #include "gdr_decode.cuh"
+#include "gdr_decode_chunk.cuh"
 #include "gdr_decode_tma.cuh"
 
 namespace {
@@ -66,6 +67,28 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   });
   return fn;
+}
+
+// The pool seen as a 3-D bf16 array [D_v / 64 column blocks][pool * H_v * D_k
+// rows][64 columns] (row stride D_v * 2 bytes, block stride 128 bytes). One
+// box {64, D_k, VS / 64} is a whole tile and lands in shared memory as
+// [block][row][64 columns] with the 128-byte swizzle: within each 128-byte
+// row segment, 16-byte chunk c is stored at position c ^ (row % 8).
+int encode_pool_map(const gdr::DecodeParams& p, int DK, int VS, CUtensorMap* map) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t gdim[3] = {64, static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK,
+                              static_cast<cuuint64_t>(p.D_v / 64)};
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(p.D_v) * 2, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(DK), static_cast<cuuint32_t>(VS / 64)};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  const CUresult cr = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                             const_cast<uint16_t*>(p.state_pool), gdim, gstride, box, estride,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  return GDR_OK;
 }
 
 constexpr int kMaxDevices = 64;
@@ -175,26 +198,9 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   const int smem = cfg.smem;
   const int ctas_per_sm = cfg.ctas_per_sm;
 
-  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-  if (encode == nullptr) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  // The pool seen as a 3-D bf16 array [D_v / 64 column blocks][pool * H_v * D_k
-  // rows][64 columns] (row stride D_v * 2 bytes, block stride 128 bytes). One
-  // box {64, D_k, VS / 64} is a whole tile and lands in shared memory as
-  // [block][row][64 columns] with the 128-byte swizzle: within each 128-byte
-  // row segment, 16-byte chunk c is stored at position c ^ (row % 8), so the
-  // consumers' 16-byte reads of different rows fall in different banks.
   CUtensorMap map;
-  const cuuint64_t gdim[3] = {64, static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK,
-                              static_cast<cuuint64_t>(p.D_v / 64)};
-  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(p.D_v) * 2, 128};
-  const cuuint32_t box[3] = {64, DK, VS / 64};
-  const cuuint32_t estride[3] = {1, 1, 1};
-  const CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                             const_cast<uint16_t*>(p.state_pool), gdim, gstride, box, estride,
-                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  rc = encode_pool_map(p, DK, VS, &map);
+  if (rc != GDR_OK) return rc;
 
   const int n_tiles = p.B * p.H_v * (p.D_v / VS);
   const int max_ctas = ctas_per_sm * props.sms;
@@ -207,19 +213,98 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   return GDR_OK;
 }
 
+// ---------------------------------------------------------------- chunk path (T >= 2)
+
+#ifndef GDR_CHUNK_MAX_STAGES
+#define GDR_CHUNK_MAX_STAGES 8
+#endif
+
+struct ChunkConfig {
+  int n_stages = 0;
+  int smem = 0;
+  int threads = 0;
+};
+
+
+// One persistent CTA per SM: as many stages as shared memory holds, and one
+// consumer group fewer than stages (so no group waits two phases ahead).
+template <int DK, int VS, bool GATED>
+int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
+  static ChunkConfig cache[kMaxDevices][gdr::kMaxT + 1];
+  static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
+  if (ready[dev][T].load(std::memory_order_acquire)) {
+    *out = cache[dev][T];
+    return GDR_OK;
+  }
+  auto kernel = gdr::decode_chunk_kernel<DK, VS, GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         props.smem_optin);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
+  constexpr int kMaxStagesChunk = GDR_CHUNK_MAX_STAGES;
+  const int stage_bytes = gdr::chunk_layout<DK, VS>(T).bytes;
+  int n = (props.smem_optin - 1024 - gdr::kChunkBarriers * 8 * kMaxStagesChunk) / stage_bytes;
+  n = n > kMaxStagesChunk ? kMaxStagesChunk : n;
+  if (n < 2) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+  constexpr int cwt = gdr::ChunkShape<DK, VS>::kWarpsPerTile;
+  int groups = n - 1;
+  const int max_groups = (gdr::kChunkMaxThreads / 32 - 2) / cwt;
+  groups = groups > max_groups ? max_groups : groups;
+  ChunkConfig c;
+  c.n_stages = n;
+  c.smem = gdr::chunk_smem_bytes<DK, VS>(T, n);
+  c.threads = 32 * (2 + groups * cwt);
+  int resident = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, c.threads, c.smem);
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(err));
+  if (resident < 1) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit on an SM");
+  cache[dev][T] = c;
+  ready[dev][T].store(true, std::memory_order_release);
+  *out = c;
+  return GDR_OK;
+}
+
+template <int DK, int VS, bool GATED>
+int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
+  DeviceProps props;
+  int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  ChunkConfig cfg;
+  rc = chunk_config<DK, VS, GATED>(dev, p.T, props, &cfg);
+  if (rc != GDR_OK) return rc;
+  CUtensorMap map;
+  rc = encode_pool_map(p, DK, VS, &map);
+  if (rc != GDR_OK) return rc;
+  const int n_tiles = p.B * p.H_v * (p.D_v / VS);
+  const int grid = n_tiles < props.sms ? n_tiles : props.sms;
+  gdr::decode_chunk_kernel<DK, VS, GATED><<<grid, cfg.threads, cfg.smem, stream>>>(map, p, n_tiles,
+                                                                                  cfg.n_stages);
+  err = cudaGetLastError();
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  return GDR_OK;
+}
+
 using LaunchFn = int (*)(const gdr::DecodeParams&, cudaStream_t);
 struct SliceKernel {
   int vs;
   LaunchFn launch;
 };
 
-// Tile widths per path, widest first, with the rows each consumer thread
-// holds. The thread count of a block caps the registers ptxas may give a
-// thread (255 up to 256 threads, 168 up to 384, 128 up to 512, 96 up to 640).
-// A single-token call keeps no state in registers (about 75 of them), so a
-// full-width 64 x 512 tile can use 16 consumer warps. A multi-token call keeps
-// fp32 state across tokens and stays within 168 (D_k = 64, 8 rows) or 255
-// (D_k = 128, 16 rows) registers.
+// Tile widths per path, widest first. Single-token calls use the
+// warp-specialised kernel with the rows each consumer thread holds; the
+// thread count of a block caps the registers ptxas may give a thread (255 up
+// to 256 threads, 168 up to 384, 128 up to 512, 96 up to 640), and a
+// single-token call keeps no state in registers (about 75 of them), so a
+// full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls use
+// the chunked kernel (64 columns per consumer warp).
 template <bool GATED>
 const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
   static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED, true>},
@@ -229,13 +314,12 @@ const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
   static const SliceKernel k128_one[] = {{256, launch_tma<128, 256, 16, GATED, true>},
                                          {128, launch_tma<128, 128, 16, GATED, true>},
                                          {64, launch_tma<128, 64, 16, GATED, true>}};
-  static const SliceKernel k64_many[] = {{256, launch_tma<64, 256, 8, GATED, false>},
-                                         {128, launch_tma<64, 128, 8, GATED, false>},
-                                         {64, launch_tma<64, 64, 8, GATED, false>}};
-  static const SliceKernel k128_many[] = {{128, launch_tma<128, 128, 16, GATED, false>},
-                                          {64, launch_tma<128, 64, 16, GATED, false>}};
+  static const SliceKernel k64_many[] = {{128, launch_chunk<64, 128, GATED>},
+                                         {64, launch_chunk<64, 64, GATED>}};
+  static const SliceKernel k128_many[] = {{128, launch_chunk<128, 128, GATED>},
+                                          {64, launch_chunk<128, 64, GATED>}};
   if (D_k == 64) {
-    *n = one ? 4 : 3;
+    *n = one ? 4 : 2;
     return one ? k64_one : k64_many;
   }
   *n = one ? 3 : 2;

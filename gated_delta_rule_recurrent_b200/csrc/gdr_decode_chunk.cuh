@@ -1,0 +1,695 @@
+// Multi-token decode kernel (T >= 2) for sm_100a: all L tokens of an item in
+// one pass over the state.
+//
+// Arithmetic: the four steps of "lite_boost.ops.recurrent_gated_delta_rule"
+// (MindSpore Lite API page, section 算法流程), applied to tokens t = 0..L-1 of
+// one (item, value head), and, when GATED, the gate of
+// "com.microsoft.LinearAttentionGate" (README, section Description).
+//
+// Write d_t = exp(g_t + gk_t) (a D_k vector), D_t = diag(d_t), q^_t = q_t *
+// scale, and for s <= t the decay products P_t = D_0 ... D_t and
+// P_{s->t} = D_{s+1} ... D_t (the identity when s = t). Unrolling the
+// recurrence S_t = D_t S_{t-1} + k_t delta_t^T from the loaded state S_0:
+//
+//   S_t            = P_t S_0 + sum_{s<=t} P_{s->t} k_s delta_s^T
+//   kv_mem_t       = (D_t S_{t-1})^T k_t = S_0^T u_t + sum_{s<t} A_ts delta_s
+//   o_t            = S_t^T q^_t          = S_0^T w_t + sum_{s<=t} B_ts delta_s
+//   delta_t        = beta_t (v_t - kv_mem_t)
+//
+// with u_t = P_t k_t, w_t = P_t q^_t, A_ts = k_s . (P_{s->t} k_t) and
+// B_ts = k_s . (P_{s->t} q^_t). The new state is S_L = c o S_0 + sum_s e_s
+// delta_s^T with c = P_{L-1} (per row) and e_s = P_{s->L-1} k_s. These are the
+// same sums as the token-by-token recurrence, regrouped; only the rounding
+// order differs. The products P_{s->t} are built by running multiplication
+// (never by division), so no intermediate can overflow when the decays are
+// small.
+//
+// A tile is one (item b, value head h, VS-column slice) of the state. Each CTA
+// walks tiles blockIdx.x, + gridDim.x, ... through a ring of shared-memory
+// stages:
+//
+//   producer warp - starts the copies of a tile (one TMA box for the state,
+//           128-byte swizzled; one 1-D bulk copy each for the k, q and gk
+//           rows of the valid tokens, which are contiguous in HBM, and for
+//           the value rows; 4-byte cp.async copies of the gate scalars). Its
+//           lanes read the slots and lengths of the next 32 tiles ahead.
+//   marker warp - marks each tile ready, in tile order, once its copies have
+//           landed, so that readiness never waits behind the producer.
+//   consumer groups - a group of VS / 32 warps takes every NG-th tile; warp
+//           w of the group owns columns [32 w, 32 w + 32) of the tile.
+//           1. Finalise: each warp turns its own D_k / (VS / 32) rows (one
+//              per lane) into d, u, w, e and c, and its partial sums of A
+//              and B (a warp reduce-scatter into its own slot); the group
+//              meets on an mbarrier, and each warp then adds up a share of
+//              the entries in a fixed warp order (deterministic).
+//           2. Pass 1: lane (row group rg = lane / 8, column lane cl = lane %
+//              8) reads 4 columns of the row quads 4 m + rg of the bf16 state
+//              and forms the column sums S_0^T u_t and S_0^T w_t with packed
+//              fp32 pairs over (even row, odd row), at most four tokens per
+//              sweep; a reduce-scatter over the row groups leaves each lane
+//              the sums of one column.
+//           3. Each lane solves the unit lower-triangular system for delta
+//              in its column and writes o; four shuffles per token hand every
+//              lane the deltas of its 4 columns.
+//           4. Pass 2 reads the state again and writes S_L to the slot with
+//              8-byte stores.
+//
+// No step waits on another token's reduction, so the latency of a tile is one
+// pass of sums, an L x L solve and one pass of updates whatever L is.
+//
+// Every mbarrier wait is bounded; a wait that runs out sets a bit in the
+// device error word and the kernel carries on with the same control flow.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdr_decode.cuh"
+#include "gdr_ptx.cuh"
+
+namespace gdr {
+
+constexpr int kChunkWarpCols = 32;      // columns per consumer warp: 8 lanes x 4
+constexpr int kChunkMaxThreads = 448;   // 12 consumer warps + the producer and marker warps
+constexpr int kChunkMaxSubTokens = 4;   // tokens per pass-1 sweep
+
+template <int DK, int VS>
+struct ChunkShape {
+  static constexpr int kWarpsPerTile = VS / kChunkWarpCols;
+  static constexpr int kStateBytes = DK * VS * 2;
+  static_assert(DK == 64 || DK == 128, "D_k must be 64 or 128");
+  static_assert(VS == 64 || VS == 128, "64- or 128-column tiles");
+};
+
+// Byte offsets inside one stage, for T padded tokens. Per-row vectors are
+// fp32 [T][DK] (token-major), so four consecutive rows of one token are one
+// 16-byte read.
+struct ChunkLayout {
+  int v, k, q, u, w, e, c, part, a, bm, beta, raw, meta, bytes;
+};
+
+template <int DK, int VS>
+__host__ __device__ inline ChunkLayout chunk_layout(int T) {
+  ChunkLayout s;
+  s.v = ChunkShape<DK, VS>::kStateBytes;  // bf16 [T][VS]  value rows of the slice
+  s.k = s.v + T * VS * 2;                 // bf16 [T][DK]  key rows
+  s.q = s.k + T * DK * 2;                 // bf16 [T][DK]  query rows
+  s.u = s.q + T * DK * 2;                 // fp32 [T][DK]  gk rows as loaded, then u_t
+  s.w = s.u + T * DK * 4;                 // fp32 [T][DK]  w_t
+  s.e = s.w + T * DK * 4;                 // fp32 [T][DK]  e_s
+  s.c = s.e + T * DK * 4;                 // fp32 [DK]     c
+  s.part = s.c + DK * 4;                  // fp32 [VS / 32][8][8] per-warp partial sums of A, B
+  s.a = s.part + (VS / kChunkWarpCols) * 256;  // fp32 [8][8]   A_ts at [t][s], s < t
+  s.bm = s.a + 256;                       // fp32 [8][8]   B_ts at [t][s], s <= t
+  s.beta = s.bm + 256;                    // fp32 [8]
+  s.raw = s.beta + 32;                    // u32 [8] g or a words, [8] beta or b words, dt_bias, decay_scale
+  s.meta = s.raw + 80;                    // int32 [4]      length, slot
+  s.bytes = (s.meta + 16 + 1023) & ~1023;
+  return s;
+}
+
+// Five mbarriers per stage: copies landed, tile ready, row vectors written,
+// A and B summed, stage released.
+constexpr int kChunkBarriers = 5;
+template <int DK, int VS>
+__host__ __device__ inline int chunk_smem_bytes(int T, int n_stages) {
+  return 1024 /* alignment slack */ + n_stages * chunk_layout<DK, VS>(T).bytes +
+         kChunkBarriers * n_stages * 8;
+}
+
+// In-register butterfly reduce-scatter of N values (N a power of two) over the
+// 32 lanes of a warp. On return lane holds n = max(N / 32, 1) totals in
+// v[0 .. n), the totals of entries base + [0, n) with base from
+// reduce_scatter_base<N>(lane). For N < 32 the same total sits in 32 / N
+// lanes; the one with reduce_scatter_writer<N>(lane) stores it.
+template <int N, int BIT>
+__device__ __forceinline__ void reduce_scatter_level(float (&v)[N], int lane) {
+  constexpr int n = N >> (BIT == 16 ? 0 : BIT == 8 ? 1 : BIT == 4 ? 2 : BIT == 2 ? 3 : 4);
+  if constexpr (n >= 2) {
+    constexpr int H = n / 2;
+    const bool up = (lane & BIT) != 0;
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+      const float send = up ? v[i] : v[i + H];
+      const float keep = up ? v[i + H] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, BIT);
+    }
+  } else {
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], BIT);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void reduce_scatter(float (&v)[N], int lane) {
+  reduce_scatter_level<N, 16>(v, lane);
+  reduce_scatter_level<N, 8>(v, lane);
+  reduce_scatter_level<N, 4>(v, lane);
+  reduce_scatter_level<N, 2>(v, lane);
+  reduce_scatter_level<N, 1>(v, lane);
+}
+
+template <int N>
+__device__ __forceinline__ int reduce_scatter_base(int lane) {
+  int base = 0, n = N;
+#pragma unroll
+  for (int bit = 16; bit >= 1; bit >>= 1) {
+    if (n >= 2) {
+      n >>= 1;
+      if (lane & bit) base += n;
+    }
+  }
+  return base;
+}
+
+template <int N>
+__device__ __forceinline__ bool reduce_scatter_writer(int lane) {
+  return N >= 32 ? true : (lane & (32 / N - 1)) == 0;
+}
+
+constexpr int pow2_at_least(int x) {
+  int n = 1;
+  while (n < x) n <<= 1;
+  return n;
+}
+
+// bf16 state words of rows (i, i + 1), 4 columns each, as packed fp32 pairs
+// over the two rows: x[c] = {S[i][c0 + c], S[i + 1][c0 + c]}.
+__device__ __forceinline__ void row_pair_columns(const uint2 a, const uint2 b,
+                                                 unsigned long long (&x)[4]) {
+  x[0] = pk(bf16_lo(a.x), bf16_lo(b.x));
+  x[1] = pk(bf16_hi(a.x), bf16_hi(b.x));
+  x[2] = pk(bf16_lo(a.y), bf16_lo(b.y));
+  x[3] = pk(bf16_hi(a.y), bf16_hi(b.y));
+}
+
+// The 8 bytes of columns [c0, c0 + 4) of row i in a swizzled state tile.
+template <int DK>
+__device__ __forceinline__ uint2 state_quad(const uint8_t* st, int i, int c0) {
+  return *reinterpret_cast<const uint2*>(st + swz_offset<DK>(i, c0) + (c0 & 7) * 2);
+}
+
+// Which of a lane's 4 columns it solves for, by row group: the reduce-scatter
+// first splits the columns by row-group bit 0, then by bit 1.
+__device__ __forceinline__ int solved_column(int rg) { return 2 * (rg & 1) + (rg >> 1); }
+// The row group that solves column j of a lane's 4 (the inverse map).
+__device__ __forceinline__ int solver_group(int j) { return (j & 1) * 2 + (j >> 1); }
+
+// ---------------------------------------------------------------- finalise
+
+// Row vectors and this warp's partial sums of A and B for a tile with L = LC
+// tokens. Warp gw of the group takes rows gw * 32 + lane + 32 * CWT * k; the
+// gate value g_t sits in lane t (t < LC). The partial sums go to this warp's
+// own [8][8] slot (entry (r, col): B_{t=r, s=col} for col <= r, A_{t=col,
+// s=r} for col > r); chunk_sum_parts adds the slots in a fixed order.
+template <int DK, int CWT, int LC>
+__device__ __forceinline__ void chunk_finalize(uint8_t* st, const ChunkLayout& lay, float g_lane,
+                                               float scale, int lane, int gw) {
+  constexpr int NM = pow2_at_least(LC * LC);  // partial sums, padded for the reduce-scatter
+  float g[LC];
+#pragma unroll
+  for (int t = 0; t < LC; ++t) g[t] = __shfl_sync(0xffffffffu, g_lane, t);
+  const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);  // [T][DK]
+  const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
+  float* su = reinterpret_cast<float*>(st + lay.u);
+  float* sw = reinterpret_cast<float*>(st + lay.w);
+  float* se = reinterpret_cast<float*>(st + lay.e);
+  float* sc = reinterpret_cast<float*>(st + lay.c);
+  // mp[s * LC + t] (s < t) holds A_ts, mp[t * LC + s] (s <= t) holds B_ts
+  float mp[NM];
+#pragma unroll
+  for (int i = 0; i < NM; ++i) mp[i] = 0.0f;
+#pragma unroll 1
+  for (int i = gw * 32 + lane; i < DK; i += 32 * CWT) {
+    float d[LC], kf[LC], qf[LC];
+#pragma unroll
+    for (int t = 0; t < LC; ++t) {
+      d[t] = expf(g[t] + su[t * DK + i]);  // exp(g) * exp(gk) as one exponential
+      kf[t] = bf16_bits_to_f32(sk[t * DK + i]);
+      qf[t] = bf16_bits_to_f32(sq[t * DK + i]) * scale;
+    }
+    float P = 1.0f;
+#pragma unroll
+    for (int t = 0; t < LC; ++t) {
+      P = t == 0 ? d[0] : P * d[t];
+      su[t * DK + i] = P * kf[t];  // u_t over the gk entry just read
+      sw[t * DK + i] = P * qf[t];
+    }
+    sc[i] = P;
+#pragma unroll
+    for (int s = 0; s < LC; ++s) {
+      float z = kf[s];  // P_{s->t} k_s by running products
+      mp[s * LC + s] = fmaf(z, qf[s], mp[s * LC + s]);
+#pragma unroll
+      for (int t = s + 1; t < LC; ++t) {
+        z *= d[t];
+        mp[s * LC + t] = fmaf(z, kf[t], mp[s * LC + t]);
+        mp[t * LC + s] = fmaf(z, qf[t], mp[t * LC + s]);
+      }
+      se[s * DK + i] = z;
+    }
+  }
+  reduce_scatter<NM>(mp, lane);
+  constexpr int NL = NM >= 32 ? NM / 32 : 1;
+  if (reduce_scatter_writer<NM>(lane)) {
+    const int base = reduce_scatter_base<NM>(lane);
+    float* part = reinterpret_cast<float*>(st + lay.part) + gw * 64;
+#pragma unroll
+    for (int j = 0; j < NL; ++j) {
+      const int f = base + j;
+      if (f < LC * LC) part[(f / LC) * 8 + f % LC] = mp[j];
+    }
+  }
+}
+
+// A and B from the group's partial sums, in warp order: warp gw of the group
+// sums the entries [gw * 64 / CWT, (gw + 1) * 64 / CWT) of the [8][8] grid.
+template <int CWT>
+__device__ __forceinline__ void chunk_sum_parts(uint8_t* st, const ChunkLayout& lay, int L,
+                                                int lane, int gw) {
+  constexpr int PER = 64 / CWT;
+  if (lane < PER) {
+    const int f = gw * PER + lane;
+    const int r = f >> 3, col = f & 7;
+    if (r < L && col < L) {
+      const float* part = reinterpret_cast<const float*>(st + lay.part);
+      float x = part[f];
+#pragma unroll
+      for (int w = 1; w < CWT; ++w) x += part[w * 64 + f];
+      if (col > r) reinterpret_cast<float*>(st + lay.a)[col * 8 + r] = x;  // A_{t = col, s = r}
+      else reinterpret_cast<float*>(st + lay.bm)[f] = x;                   // B_{t = r, s = col}
+    }
+  }
+}
+
+template <int DK, int CWT>
+__device__ __forceinline__ void chunk_finalize_any(int L, uint8_t* st, const ChunkLayout& lay,
+                                                   float g_lane, float scale, int lane, int gw) {
+  switch (L) {
+    case 1: chunk_finalize<DK, CWT, 1>(st, lay, g_lane, scale, lane, gw); break;
+    case 2: chunk_finalize<DK, CWT, 2>(st, lay, g_lane, scale, lane, gw); break;
+    case 3: chunk_finalize<DK, CWT, 3>(st, lay, g_lane, scale, lane, gw); break;
+    case 4: chunk_finalize<DK, CWT, 4>(st, lay, g_lane, scale, lane, gw); break;
+    case 5: chunk_finalize<DK, CWT, 5>(st, lay, g_lane, scale, lane, gw); break;
+    case 6: chunk_finalize<DK, CWT, 6>(st, lay, g_lane, scale, lane, gw); break;
+    case 7: chunk_finalize<DK, CWT, 7>(st, lay, g_lane, scale, lane, gw); break;
+    case 8: chunk_finalize<DK, CWT, 8>(st, lay, g_lane, scale, lane, gw); break;
+    default: break;
+  }
+}
+
+// ---------------------------------------------------------------- consumers
+
+// Pass-1 sweep over tokens [T0, T0 + LS) of a tile: the column sums
+// S_0^T u_t and S_0^T w_t of this lane's solved column into ms[t], ps[t].
+template <int DK, int LC, int T0, int LS>
+__device__ __forceinline__ void chunk_sums(const uint8_t* st, const float* su, const float* sw,
+                                           int c0, int rg, int lane, float (&ms)[LC],
+                                           float (&ps)[LC]) {
+  unsigned long long acc[2 * LS][4];
+#pragma unroll
+  for (int v = 0; v < 2 * LS; ++v)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[v][c] = 0ull;  // (+0.0f, +0.0f)
+#pragma unroll 1
+  for (int m = 0; m < DK / 16; ++m) {
+    const int r0 = 16 * m + 4 * rg;
+    unsigned long long x0[4], x1[4];
+    row_pair_columns(state_quad<DK>(st, r0, c0), state_quad<DK>(st, r0 + 1, c0), x0);
+    row_pair_columns(state_quad<DK>(st, r0 + 2, c0), state_quad<DK>(st, r0 + 3, c0), x1);
+#pragma unroll
+    for (int t = 0; t < LS; ++t) {
+      const ulonglong2 uq = *reinterpret_cast<const ulonglong2*>(su + (T0 + t) * DK + r0);
+      const ulonglong2 wq = *reinterpret_cast<const ulonglong2*>(sw + (T0 + t) * DK + r0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[t][c] = fma2(x0[c], uq.x, acc[t][c]);
+        acc[LS + t][c] = fma2(x0[c], wq.x, acc[LS + t][c]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[t][c] = fma2(x1[c], uq.y, acc[t][c]);
+        acc[LS + t][c] = fma2(x1[c], wq.y, acc[LS + t][c]);
+      }
+    }
+  }
+  // fold (even row, odd row), then reduce-scatter over the row groups: lane
+  // bit 3 keeps columns {2, 3} or {0, 1}, lane bit 4 one of those two
+  const bool b0 = (lane >> 3) & 1, b1 = (lane >> 4) & 1;
+#pragma unroll
+  for (int v = 0; v < 2 * LS; ++v) {
+    float y[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float2 a = upk(acc[v][c]);
+      y[c] = a.x + a.y;
+    }
+    float z[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float send = b0 ? y[j] : y[j + 2];
+      const float keep = b0 ? y[j + 2] : y[j];
+      z[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const float send = b1 ? z[0] : z[1];
+    const float keep = b1 ? z[1] : z[0];
+    const float f = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    if (v < LS) ms[T0 + v] = f;
+    else ps[T0 + v - LS] = f;
+  }
+}
+
+// One tile with L = LC tokens, for one consumer warp (columns [c0, c0 + 4)
+// of the tile in this lane). `dst` points at row 0, column c0 of the slot's
+// slice; `out_t0` at token 0, column 0 of the tile's output.
+template <int DK, int VS, int LC>
+__device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayout& lay, int c0,
+                                              int rg, int lane, uint16_t* dst, uint16_t* out_t0,
+                                              int D_v, uint32_t sum_bar, uint32_t phase) {
+  const float* su = reinterpret_cast<const float*>(st + lay.u);
+  const float* sw = reinterpret_cast<const float*>(st + lay.w);
+  const float* se = reinterpret_cast<const float*>(st + lay.e);
+  const float* sc = reinterpret_cast<const float*>(st + lay.c);
+
+  // ---- pass 1: column sums, at most four tokens per sweep of the state
+  float ms[LC], ps[LC];
+  chunk_sums<DK, LC, 0, (LC < kChunkMaxSubTokens ? LC : kChunkMaxSubTokens)>(st, su, sw, c0, rg,
+                                                                            lane, ms, ps);
+  if constexpr (LC > kChunkMaxSubTokens)
+    chunk_sums<DK, LC, kChunkMaxSubTokens, LC - kChunkMaxSubTokens>(st, su, sw, c0, rg, lane, ms,
+                                                                   ps);
+
+  // ---- delta (unit lower-triangular solve) and o, for the solved column
+  if (!mbar_wait_bounded(sum_bar, phase)) flag_error(kErrConsumerWait);  // A and B summed
+  const int col = c0 + solved_column(rg);
+  const float* sa = reinterpret_cast<const float*>(st + lay.a);
+  const float* sb = reinterpret_cast<const float*>(st + lay.bm);
+  const float* sbeta = reinterpret_cast<const float*>(st + lay.beta);
+  const uint16_t* sv = reinterpret_cast<const uint16_t*>(st + lay.v);
+  float dl[LC];
+#pragma unroll
+  for (int t = 0; t < LC; ++t) {
+    float kv = ms[t];  // kv_mem_t = S_0^T u_t + sum_{s<t} A_ts delta_s
+#pragma unroll
+    for (int s = 0; s < t; ++s) kv = fmaf(sa[t * 8 + s], dl[s], kv);
+    dl[t] = (bf16_bits_to_f32(sv[t * VS + col]) - kv) * sbeta[t];  // step 3
+    float o = ps[t];  // o_t = S_0^T w_t + sum_{s<=t} B_ts delta_s (step 4)
+#pragma unroll
+    for (int s = 0; s <= t; ++s) o = fmaf(sb[t * 8 + s], dl[s], o);
+    out_t0[static_cast<size_t>(t) * D_v + col] = f32_to_bf16_bits(o);
+  }
+  // every lane gathers the deltas of its 4 columns: {delta_s[c], delta_s[c]}
+  const int cl = lane & 7;
+  unsigned long long dd[LC][4];
+#pragma unroll
+  for (int s = 0; s < LC; ++s)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x = __shfl_sync(0xffffffffu, dl[s], solver_group(j) * 8 + cl);
+      dd[s][j] = pk(x, x);
+    }
+
+  // ---- pass 2: S_L = c o S_0 + sum_s e_s delta_s^T, bf16 once, to the slot
+#pragma unroll 1
+  for (int m = 0; m < DK / 16; ++m) {
+    const int r0 = 16 * m + 4 * rg;
+    unsigned long long n0[4], n1[4];
+    row_pair_columns(state_quad<DK>(st, r0, c0), state_quad<DK>(st, r0 + 1, c0), n0);
+    row_pair_columns(state_quad<DK>(st, r0 + 2, c0), state_quad<DK>(st, r0 + 3, c0), n1);
+    const ulonglong2 cq = *reinterpret_cast<const ulonglong2*>(sc + r0);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      n0[c] = mul2(n0[c], cq.x);
+      n1[c] = mul2(n1[c], cq.y);
+    }
+#pragma unroll
+    for (int s = 0; s < LC; ++s) {
+      const ulonglong2 eq = *reinterpret_cast<const ulonglong2*>(se + s * DK + r0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        n0[c] = fma2(eq.x, dd[s][c], n0[c]);
+        n1[c] = fma2(eq.y, dd[s][c], n1[c]);
+      }
+    }
+    float2 a[4], b[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      a[c] = upk(n0[c]);
+      b[c] = upk(n1[c]);
+    }
+    uint16_t* d0 = dst + static_cast<size_t>(r0) * D_v;
+    __stcs(reinterpret_cast<uint2*>(d0),
+           make_uint2(pack_bf16x2(a[0].x, a[1].x), pack_bf16x2(a[2].x, a[3].x)));
+    __stcs(reinterpret_cast<uint2*>(d0 + D_v),
+           make_uint2(pack_bf16x2(a[0].y, a[1].y), pack_bf16x2(a[2].y, a[3].y)));
+    __stcs(reinterpret_cast<uint2*>(d0 + 2 * D_v),
+           make_uint2(pack_bf16x2(b[0].x, b[1].x), pack_bf16x2(b[2].x, b[3].x)));
+    __stcs(reinterpret_cast<uint2*>(d0 + 3 * D_v),
+           make_uint2(pack_bf16x2(b[0].y, b[1].y), pack_bf16x2(b[2].y, b[3].y)));
+  }
+}
+
+template <int DK, int VS>
+__device__ __forceinline__ void chunk_consume_any(int L, const uint8_t* st, const ChunkLayout& lay,
+                                                  int c0, int rg, int lane, uint16_t* dst,
+                                                  uint16_t* out_t0, int D_v, uint32_t sum_bar,
+                                                  uint32_t phase) {
+  switch (L) {
+    case 1: chunk_consume<DK, VS, 1>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 2: chunk_consume<DK, VS, 2>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 3: chunk_consume<DK, VS, 3>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 4: chunk_consume<DK, VS, 4>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 5: chunk_consume<DK, VS, 5>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 6: chunk_consume<DK, VS, 6>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 7: chunk_consume<DK, VS, 7>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 8: chunk_consume<DK, VS, 8>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    default: break;
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+// Block: NG groups of VS / 32 consumer warps, then the marker and producer
+// warps; NG = (blockDim.x / 32 - 2) / (VS / 32). Requires n_stages >= NG + 1:
+// tiles are marked ready in order, so a group never waits on a stage two
+// phases ahead of it.
+template <int DK, int VS, bool GATED>
+__global__ void __launch_bounds__(kChunkMaxThreads, 1)
+    decode_chunk_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
+                        const int n_tiles, const int n_stages) {
+  using Shape = ChunkShape<DK, VS>;
+  constexpr int CWT = Shape::kWarpsPerTile;
+  const int T = p.T;
+  const ChunkLayout lay = chunk_layout<DK, VS>(T);
+
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t raw_base = smem_addr(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + n_stages * lay.bytes);
+  const uint32_t raw0 = smem_addr(bars);         // copies landed
+  const uint32_t full0 = raw0 + 8 * n_stages;    // tile ready (in tile order)
+  const uint32_t fin0 = full0 + 8 * n_stages;    // the group's row vectors are written
+  const uint32_t sum0 = fin0 + 8 * n_stages;     // the group's A and B are summed
+  const uint32_t empty0 = sum0 + 8 * n_stages;   // the group is done with the stage
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int producer = static_cast<int>(blockDim.x >> 5) - 1;
+  const int marker = producer - 1;
+  const int n_groups = marker / CWT;
+  const int n_slices = p.D_v / VS;
+  const int n_mine = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                     static_cast<int>(gridDim.x);
+
+  if (tid == 0) {
+    for (int i = 0; i < n_stages; ++i) {
+      mbar_init(raw0 + 8 * i, 32);     // one cp.async arrival per producer lane
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(fin0 + 8 * i, CWT);    // one arrival per warp of the group
+      mbar_init(sum0 + 8 * i, CWT);
+      mbar_init(empty0 + 8 * i, CWT);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == marker) {
+    // ================================================================ marker
+    // Tiles become ready in tile order; so a group that waits for tile x
+    // finds the stage's barrier at tile x's phase (tile x - n_stages was
+    // marked before it). Waiting on every tile's copies also means the CTA
+    // never retires with copies in flight.
+    if (lane == 0) {
+      for (int j = 0; j < n_mine; ++j) {
+        const int stage = j % n_stages;
+        if (!mbar_wait_bounded(raw0 + 8 * stage, (j / n_stages) & 1)) flag_error(kErrProducerWait);
+        mbar_arrive(full0 + 8 * stage);
+      }
+    }
+    return;
+  }
+  if (warp == producer) {
+    // ================================================================ producer
+    bool failed = false;
+    // lane i holds the slot and length of tile (j & ~31) + i; the next 32
+    // tiles' are loaded 32 tiles ahead
+    auto load_index = [&](int jj, int& slot, int& len) {
+      slot = 0;
+      len = 0;
+      if (jj < n_mine) {
+        const int bb = (blockIdx.x + jj * gridDim.x) / (n_slices * p.H_v);
+        slot = p.state_indices[bb];
+        len = p.seq_lengths[bb];
+      }
+    };
+    int cur_s, cur_L, nxt_s, nxt_L;
+    load_index(lane, cur_s, cur_L);
+    load_index(32 + lane, nxt_s, nxt_L);
+    for (int j = 0; j < n_mine; ++j) {
+      if (j > 0 && (j & 31) == 0) {
+        cur_s = nxt_s;
+        cur_L = nxt_L;
+        load_index(j + 32 + lane, nxt_s, nxt_L);
+      }
+      const int tile = blockIdx.x + j * gridDim.x;
+      const int slice = tile % n_slices;
+      const int h = (tile / n_slices) % p.H_v;
+      const int b = tile / (n_slices * p.H_v);
+      const int s = __shfl_sync(0xffffffffu, cur_s, j & 31);
+      int L = __shfl_sync(0xffffffffu, cur_L, j & 31);
+      L = L < 0 ? 0 : (L > T ? T : L);
+      if (s < 0 || s >= p.pool_size) L = 0;
+      const int stage = j % n_stages;
+      const uint32_t phase = (j / n_stages) & 1;
+      uint8_t* st = smem + stage * lay.bytes;
+      const uint32_t rawb = raw0 + 8 * stage;
+      if (lane == 0 && !failed) {
+        if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1)) {
+          failed = true;
+          flag_error(kErrProducerWait);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        int* meta = reinterpret_cast<int*>(st + lay.meta);
+        meta[0] = L;
+        meta[1] = s;
+        if (L > 0) {
+          mbar_expect_tx(rawb, Shape::kStateBytes + L * (VS * 2 + DK * 8));
+          // the L valid tokens' rows are contiguous in HBM: one copy each
+          const int col0 = slice * VS;
+          const size_t qk_off = (static_cast<size_t>(b) * p.H_qk + h / p.group) * T * DK;
+          const size_t gk_off = (static_cast<size_t>(b) * p.H_v + h) * T * DK;
+          const uint16_t* vsrc = p.value + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + col0;
+          tma_load_3d(smem_addr(st), &pool_map, 0, (s * p.H_v + h) * DK, col0 / 64, rawb);
+          bulk_load(smem_addr(st + lay.k), p.key + qk_off, L * DK * 2, rawb);
+          bulk_load(smem_addr(st + lay.q), p.query + qk_off, L * DK * 2, rawb);
+          bulk_load(smem_addr(st + lay.u), p.gk + gk_off, L * DK * 4, rawb);
+          if (VS == p.D_v) {
+            bulk_load(smem_addr(st + lay.v), vsrc, L * VS * 2, rawb);
+          } else {
+            for (int t = 0; t < L; ++t)
+              bulk_load(smem_addr(st + lay.v + t * VS * 2), vsrc + static_cast<size_t>(t) * p.D_v,
+                        VS * 2, rawb);
+          }
+        }
+      }
+      // gate scalars: lane t fetches token t's pair; lane 31 the per-head values
+      uint32_t* rawv = reinterpret_cast<uint32_t*>(st + lay.raw);
+      if (lane < L) {
+        if constexpr (GATED) {
+          const size_t ai = (static_cast<size_t>(b) * T + lane) * p.H_v + h;
+          cp_async_4(smem_addr(rawv + lane), word_of(p.gate_a + ai));
+          cp_async_4(smem_addr(rawv + 8 + lane), word_of(p.gate_b + ai));
+        } else {
+          const size_t gi = (static_cast<size_t>(b) * p.H_v + h) * T + lane;
+          cp_async_4(smem_addr(rawv + lane), p.g + gi);
+          cp_async_4(smem_addr(rawv + 8 + lane), word_of(p.beta + gi));
+        }
+      }
+      if constexpr (GATED) {
+        if (lane == 31 && L > 0) {
+          cp_async_4(smem_addr(rawv + 16), p.dt_bias + h);
+          cp_async_4(smem_addr(rawv + 17), p.decay_scale + h);
+        }
+      }
+      cp_async_arrive_noinc(rawb);
+    }
+    return;
+  }
+
+  // ================================================================ consumers
+  const int group = warp / CWT;
+  if (group >= n_groups) return;  // (no such warps with the launch shapes used)
+  const int gw = warp % CWT;
+  const int rg = lane >> 3;
+  const int c0 = gw * kChunkWarpCols + (lane & 7) * 4;  // first tile column of this lane
+  for (int it = group; it < n_mine; it += n_groups) {
+    const int tile = blockIdx.x + it * gridDim.x;
+    const int slice = tile % n_slices;
+    const int h = (tile / n_slices) % p.H_v;
+    const int b = tile / (n_slices * p.H_v);
+    const int stage = it % n_stages;
+    const uint32_t phase = (it / n_stages) & 1;
+    uint8_t* st = smem + stage * lay.bytes;
+
+    const bool ok_self = mbar_wait_bounded(full0 + 8 * stage, phase);
+    const bool ok = __all_sync(0xffffffffu, ok_self);
+    if (!ok_self) flag_error(kErrConsumerWait);
+    const int* meta = reinterpret_cast<const int*>(st + lay.meta);
+    int L = ok ? meta[0] : 0;
+    L = L < 0 ? 0 : (L > T ? T : L);
+    const int s = meta[1];
+    if (s < 0 || s >= p.pool_size) L = 0;
+
+    // out[b, h, t, slice * VS + column]; padded tokens get +0.0
+    uint16_t* out_t0 = p.out + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + slice * VS;
+    const int col = c0 + solved_column(rg);
+    for (int t = L; t < T; ++t) out_t0[static_cast<size_t>(t) * p.D_v + col] = 0;
+
+    if (L > 0) {
+      // ---- gate (lane t: token t), then this warp's rows of the finalise step
+      float gt = 0.0f;
+      if (lane < L) {
+        const uint32_t* rawv = reinterpret_cast<const uint32_t*>(st + lay.raw);
+        float bt;
+        if constexpr (GATED) {
+          const size_t ai = (static_cast<size_t>(b) * T + lane) * p.H_v + h;
+          const float dtb = __uint_as_float(rawv[16]);
+          const float dsc = __uint_as_float(rawv[17]);
+          gt = dsc * softplus_f32(bf16_in_word(rawv[lane], p.gate_a + ai) + dtb);  // g
+          bt = sigmoid_f32(bf16_in_word(rawv[8 + lane], p.gate_b + ai));          // beta
+        } else {
+          const size_t gi = (static_cast<size_t>(b) * p.H_v + h) * T + lane;
+          gt = __uint_as_float(rawv[lane]);
+          bt = bf16_in_word(rawv[8 + lane], p.beta + gi);
+        }
+        if (gw == 0) reinterpret_cast<float*>(st + lay.beta)[lane] = bt;
+      }
+      chunk_finalize_any<DK, CWT>(L, st, lay, gt, p.scale, lane, gw);
+    }
+    // The group meets twice: once the row vectors and partial sums are
+    // written, and once A and B are summed (waited for only after pass 1).
+    // Every warp arrives on both, so the phases stay in step.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(fin0 + 8 * stage);
+    if (L > 0) {
+      if (!mbar_wait_bounded(fin0 + 8 * stage, phase)) flag_error(kErrConsumerWait);
+      chunk_sum_parts<CWT>(st, lay, L, lane, gw);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sum0 + 8 * stage);
+    if (L > 0) {
+      uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
+                      slice * VS + c0;
+      chunk_consume_any<DK, VS>(L, st, lay, c0, rg, lane, dst, out_t0, p.D_v, sum0 + 8 * stage,
+                                phase);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+  }
+}
+
+}  // namespace gdr
