@@ -245,18 +245,18 @@ int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
   constexpr int kMaxStagesChunk = GDR_CHUNK_MAX_STAGES;
-  const int stage_bytes = gdr::chunk_layout<DK, VS>(T).bytes;
+  const int stage_bytes = gdr::chunk_stage_bytes<DK, VS>(T);
   int n = (props.smem_optin - 1024 - gdr::kChunkBarriers * 8 * kMaxStagesChunk) / stage_bytes;
   n = n > kMaxStagesChunk ? kMaxStagesChunk : n;
   if (n < 2) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
   constexpr int cwt = gdr::ChunkShape<DK, VS>::kWarpsPerTile;
   int groups = n - 1;
-  const int max_groups = (gdr::kChunkMaxThreads / 32 - 2) / cwt;
+  const int max_groups = (gdr::kChunkMaxThreads / 32 - 1 - gdr::kChunkFinalizers) / cwt;
   groups = groups > max_groups ? max_groups : groups;
   ChunkConfig c;
   c.n_stages = n;
   c.smem = gdr::chunk_smem_bytes<DK, VS>(T, n);
-  c.threads = 32 * (2 + groups * cwt);
+  c.threads = 32 * (1 + gdr::kChunkFinalizers + groups * cwt);
   int resident = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, c.threads, c.smem);
   if (err != cudaSuccess)

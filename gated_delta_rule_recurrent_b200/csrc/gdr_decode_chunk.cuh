@@ -33,25 +33,24 @@
 //           rows of the valid tokens, which are contiguous in HBM, and for
 //           the value rows; 4-byte cp.async copies of the gate scalars). Its
 //           lanes read the slots and lengths of the next 32 tiles ahead.
-//   marker warp - marks each tile ready, in tile order, once its copies have
-//           landed, so that readiness never waits behind the producer.
+//   finaliser warps - take every tile in tile order once its copies have
+//           landed; each turns its share of the D_k rows (one per lane) into
+//           d, u, w, e and c and its partial sums of A and B (a warp
+//           reduce-scatter into its own slot); they meet on a named barrier,
+//           add the partial sums in a fixed warp order (deterministic) and
+//           mark the tile ready.
 //   consumer groups - a group of VS / 32 warps takes every NG-th tile; warp
 //           w of the group owns columns [32 w, 32 w + 32) of the tile.
-//           1. Finalise: each warp turns its own D_k / (VS / 32) rows (one
-//              per lane) into d, u, w, e and c, and its partial sums of A
-//              and B (a warp reduce-scatter into its own slot); the group
-//              meets on an mbarrier, and each warp then adds up a share of
-//              the entries in a fixed warp order (deterministic).
-//           2. Pass 1: lane (row group rg = lane / 8, column lane cl = lane %
+//           1. Pass 1: lane (row group rg = lane / 8, column lane cl = lane %
 //              8) reads 4 columns of the row quads 4 m + rg of the bf16 state
 //              and forms the column sums S_0^T u_t and S_0^T w_t with packed
 //              fp32 pairs over (even row, odd row), at most four tokens per
 //              sweep; a reduce-scatter over the row groups leaves each lane
 //              the sums of one column.
-//           3. Each lane solves the unit lower-triangular system for delta
+//           2. Each lane solves the unit lower-triangular system for delta
 //              in its column and writes o; four shuffles per token hand every
 //              lane the deltas of its 4 columns.
-//           4. Pass 2 reads the state again and writes S_L to the slot with
+//           3. Pass 2 reads the state again and writes S_L to the slot with
 //              8-byte stores.
 //
 // No step waits on another token's reduction, so the latency of a tile is one
@@ -72,7 +71,8 @@
 namespace gdr {
 
 constexpr int kChunkWarpCols = 32;      // columns per consumer warp: 8 lanes x 4
-constexpr int kChunkMaxThreads = 448;   // 12 consumer warps + the producer and marker warps
+constexpr int kChunkFinalizers = 2;     // warps that turn landed tiles into row vectors
+constexpr int kChunkMaxThreads = 480;   // 12 consumer warps, the finalisers and the producer
 constexpr int kChunkMaxSubTokens = 4;   // tokens per pass-1 sweep
 
 template <int DK, int VS>
@@ -83,39 +83,45 @@ struct ChunkShape {
   static_assert(VS == 64 || VS == 128, "64- or 128-column tiles");
 };
 
-// Byte offsets inside one stage, for T padded tokens. Per-row vectors are
-// fp32 [T][DK] (token-major), so four consecutive rows of one token are one
-// 16-byte read.
+// Shared memory: n_stages state tiles (DK x VS bf16, 128-byte swizzled, each
+// 1024-byte aligned for the swizzle), then n_stages vector blocks, then four
+// mbarriers per stage. Offsets below are within one vector block, for T
+// padded tokens. Per-row vectors are fp32 [T][DK] (token-major), so four
+// consecutive rows of one token are one 16-byte read.
 struct ChunkLayout {
-  int v, k, q, u, w, e, c, part, a, bm, beta, raw, meta, bytes;
+  int v, k, q, e, u, w, c, part, a, bm, beta, raw, meta, bytes;
 };
 
 template <int DK, int VS>
 __host__ __device__ inline ChunkLayout chunk_layout(int T) {
   ChunkLayout s;
-  s.v = ChunkShape<DK, VS>::kStateBytes;  // bf16 [T][VS]  value rows of the slice
-  s.k = s.v + T * VS * 2;                 // bf16 [T][DK]  key rows
-  s.q = s.k + T * DK * 2;                 // bf16 [T][DK]  query rows
-  s.u = s.q + T * DK * 2;                 // fp32 [T][DK]  gk rows as loaded, then u_t
-  s.w = s.u + T * DK * 4;                 // fp32 [T][DK]  w_t
-  s.e = s.w + T * DK * 4;                 // fp32 [T][DK]  e_s
-  s.c = s.e + T * DK * 4;                 // fp32 [DK]     c
-  s.part = s.c + DK * 4;                  // fp32 [VS / 32][8][8] per-warp partial sums of A, B
-  s.a = s.part + (VS / kChunkWarpCols) * 256;  // fp32 [8][8]   A_ts at [t][s], s < t
-  s.bm = s.a + 256;                       // fp32 [8][8]   B_ts at [t][s], s <= t
-  s.beta = s.bm + 256;                    // fp32 [8]
-  s.raw = s.beta + 32;                    // u32 [8] g or a words, [8] beta or b words, dt_bias, decay_scale
-  s.meta = s.raw + 80;                    // int32 [4]      length, slot
-  s.bytes = (s.meta + 16 + 1023) & ~1023;
+  s.v = 0;                               // bf16 [T][VS]  value rows of the slice
+  s.k = s.v + T * VS * 2;                // bf16 [T][DK]  key rows
+  s.q = s.k + T * DK * 2;                // bf16 [T][DK]  query rows
+  s.e = s.q + T * DK * 2;                // fp32 [T][DK]  e_s
+  s.u = s.e + T * DK * 4;                // fp32 [T][DK]  gk rows as loaded, then u_t
+  s.w = s.u + T * DK * 4;                // fp32 [T][DK]  w_t
+  s.c = s.w + T * DK * 4;                // fp32 [DK]     c
+  s.part = s.c + DK * 4;                 // fp32 [finalisers][8][8] partial sums of A and B
+  s.a = s.part + kChunkFinalizers * 256; // fp32 [8][8]   A_ts at [t][s], s < t
+  s.bm = s.a + 256;                      // fp32 [8][8]   B_ts at [t][s], s <= t
+  s.beta = s.bm + 256;                   // fp32 [8]
+  s.raw = s.beta + 32;                   // u32 [8] g or a words, [8] beta or b words, dt_bias, decay_scale
+  s.meta = s.raw + 80;                   // int32 [4]      length, slot
+  s.bytes = (s.meta + 16 + 15) & ~15;
   return s;
 }
 
-// Five mbarriers per stage: copies landed, tile ready, row vectors written,
-// A and B summed, stage released.
-constexpr int kChunkBarriers = 5;
+// Four mbarriers per stage: vectors landed, state landed, tile finalised
+// (in tile order), stage released.
+constexpr int kChunkBarriers = 4;
+template <int DK, int VS>
+__host__ __device__ inline int chunk_stage_bytes(int T) {
+  return ChunkShape<DK, VS>::kStateBytes + chunk_layout<DK, VS>(T).bytes;
+}
 template <int DK, int VS>
 __host__ __device__ inline int chunk_smem_bytes(int T, int n_stages) {
-  return 1024 /* alignment slack */ + n_stages * chunk_layout<DK, VS>(T).bytes +
+  return 1024 /* alignment slack */ + n_stages * chunk_stage_bytes<DK, VS>(T) +
          kChunkBarriers * n_stages * 8;
 }
 
@@ -184,11 +190,15 @@ __device__ __forceinline__ void row_pair_columns(const uint2 a, const uint2 b,
   x[3] = pk(bf16_hi(a.y), bf16_hi(b.y));
 }
 
-// The 8 bytes of columns [c0, c0 + 4) of row i in a swizzled state tile.
+// Byte offsets, in a swizzled state tile, of columns [c0, c0 + 4) of rows
+// 4 rg + r (r < 4). Rows 16 m + 4 rg + r sit 16 m * 128 bytes further on: the
+// swizzle depends only on the row modulo 8, which does not change with m.
 template <int DK>
-__device__ __forceinline__ uint2 state_quad(const uint8_t* st, int i, int c0) {
-  return *reinterpret_cast<const uint2*>(st + swz_offset<DK>(i, c0) + (c0 & 7) * 2);
+__device__ __forceinline__ void quad_offsets(int rg, int c0, int (&off)[4]) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) off[r] = swz_offset<DK>(4 * rg + r, c0) + (c0 & 7) * 2;
 }
+constexpr int kQuadStep = 16 * 128;  // bytes from row quad m to m + 1 of a row group
 
 // Which of a lane's 4 columns it solves for, by row group: the reduce-scatter
 // first splits the columns by row-group bit 0, then by bit 1.
@@ -199,29 +209,30 @@ __device__ __forceinline__ int solver_group(int j) { return (j & 1) * 2 + (j >> 
 // ---------------------------------------------------------------- finalise
 
 // Row vectors and this warp's partial sums of A and B for a tile with L = LC
-// tokens. Warp gw of the group takes rows gw * 32 + lane + 32 * CWT * k; the
-// gate value g_t sits in lane t (t < LC). The partial sums go to this warp's
-// own [8][8] slot (entry (r, col): B_{t=r, s=col} for col <= r, A_{t=col,
-// s=r} for col > r); chunk_sum_parts adds the slots in a fixed order.
-template <int DK, int CWT, int LC>
-__device__ __forceinline__ void chunk_finalize(uint8_t* st, const ChunkLayout& lay, float g_lane,
-                                               float scale, int lane, int gw) {
+// tokens, in the stage's vector block `vb`. Finaliser warp fw of NF takes rows
+// fw * 32 + lane + 32 * NF * r; the gate value g_t sits in lane t (t < LC).
+// The partial sums go to this warp's own [8][8] slot (entry (r, col):
+// B_{t=r, s=col} for col <= r, A_{t=col, s=r} for col > r); chunk_sum_parts
+// adds the slots in warp order.
+template <int DK, int NF, int LC>
+__device__ __forceinline__ void chunk_finalize(uint8_t* vb, const ChunkLayout& lay, float g_lane,
+                                               float scale, int lane, int fw) {
   constexpr int NM = pow2_at_least(LC * LC);  // partial sums, padded for the reduce-scatter
   float g[LC];
 #pragma unroll
   for (int t = 0; t < LC; ++t) g[t] = __shfl_sync(0xffffffffu, g_lane, t);
-  const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);  // [T][DK]
-  const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
-  float* su = reinterpret_cast<float*>(st + lay.u);
-  float* sw = reinterpret_cast<float*>(st + lay.w);
-  float* se = reinterpret_cast<float*>(st + lay.e);
-  float* sc = reinterpret_cast<float*>(st + lay.c);
+  const uint16_t* sk = reinterpret_cast<const uint16_t*>(vb + lay.k);  // [T][DK]
+  const uint16_t* sq = reinterpret_cast<const uint16_t*>(vb + lay.q);
+  float* su = reinterpret_cast<float*>(vb + lay.u);
+  float* sw = reinterpret_cast<float*>(vb + lay.w);
+  float* se = reinterpret_cast<float*>(vb + lay.e);
+  float* sc = reinterpret_cast<float*>(vb + lay.c);
   // mp[s * LC + t] (s < t) holds A_ts, mp[t * LC + s] (s <= t) holds B_ts
   float mp[NM];
 #pragma unroll
-  for (int i = 0; i < NM; ++i) mp[i] = 0.0f;
+  for (int j = 0; j < NM; ++j) mp[j] = 0.0f;
 #pragma unroll 1
-  for (int i = gw * 32 + lane; i < DK; i += 32 * CWT) {
+  for (int i = fw * 32 + lane; i < DK; i += 32 * NF) {
     float d[LC], kf[LC], qf[LC];
 #pragma unroll
     for (int t = 0; t < LC; ++t) {
@@ -254,7 +265,7 @@ __device__ __forceinline__ void chunk_finalize(uint8_t* st, const ChunkLayout& l
   constexpr int NL = NM >= 32 ? NM / 32 : 1;
   if (reduce_scatter_writer<NM>(lane)) {
     const int base = reduce_scatter_base<NM>(lane);
-    float* part = reinterpret_cast<float*>(st + lay.part) + gw * 64;
+    float* part = reinterpret_cast<float*>(vb + lay.part) + fw * 64;
 #pragma unroll
     for (int j = 0; j < NL; ++j) {
       const int f = base + j;
@@ -263,38 +274,38 @@ __device__ __forceinline__ void chunk_finalize(uint8_t* st, const ChunkLayout& l
   }
 }
 
-// A and B from the group's partial sums, in warp order: warp gw of the group
-// sums the entries [gw * 64 / CWT, (gw + 1) * 64 / CWT) of the [8][8] grid.
-template <int CWT>
-__device__ __forceinline__ void chunk_sum_parts(uint8_t* st, const ChunkLayout& lay, int L,
-                                                int lane, int gw) {
-  constexpr int PER = 64 / CWT;
+// A and B from the finalisers' partial sums, in warp order: warp fw of NF
+// sums the entries [fw * 64 / NF, (fw + 1) * 64 / NF) of the [8][8] grid.
+template <int NF>
+__device__ __forceinline__ void chunk_sum_parts(uint8_t* vb, const ChunkLayout& lay, int L,
+                                                int lane, int fw) {
+  constexpr int PER = 64 / NF;
   if (lane < PER) {
-    const int f = gw * PER + lane;
+    const int f = fw * PER + lane;
     const int r = f >> 3, col = f & 7;
     if (r < L && col < L) {
-      const float* part = reinterpret_cast<const float*>(st + lay.part);
+      const float* part = reinterpret_cast<const float*>(vb + lay.part);
       float x = part[f];
 #pragma unroll
-      for (int w = 1; w < CWT; ++w) x += part[w * 64 + f];
-      if (col > r) reinterpret_cast<float*>(st + lay.a)[col * 8 + r] = x;  // A_{t = col, s = r}
-      else reinterpret_cast<float*>(st + lay.bm)[f] = x;                   // B_{t = r, s = col}
+      for (int w = 1; w < NF; ++w) x += part[w * 64 + f];
+      if (col > r) reinterpret_cast<float*>(vb + lay.a)[col * 8 + r] = x;  // A_{t = col, s = r}
+      else reinterpret_cast<float*>(vb + lay.bm)[f] = x;                   // B_{t = r, s = col}
     }
   }
 }
 
-template <int DK, int CWT>
-__device__ __forceinline__ void chunk_finalize_any(int L, uint8_t* st, const ChunkLayout& lay,
-                                                   float g_lane, float scale, int lane, int gw) {
+template <int DK, int NF>
+__device__ __forceinline__ void chunk_finalize_any(int L, uint8_t* vb, const ChunkLayout& lay,
+                                                   float g_lane, float scale, int lane, int fw) {
   switch (L) {
-    case 1: chunk_finalize<DK, CWT, 1>(st, lay, g_lane, scale, lane, gw); break;
-    case 2: chunk_finalize<DK, CWT, 2>(st, lay, g_lane, scale, lane, gw); break;
-    case 3: chunk_finalize<DK, CWT, 3>(st, lay, g_lane, scale, lane, gw); break;
-    case 4: chunk_finalize<DK, CWT, 4>(st, lay, g_lane, scale, lane, gw); break;
-    case 5: chunk_finalize<DK, CWT, 5>(st, lay, g_lane, scale, lane, gw); break;
-    case 6: chunk_finalize<DK, CWT, 6>(st, lay, g_lane, scale, lane, gw); break;
-    case 7: chunk_finalize<DK, CWT, 7>(st, lay, g_lane, scale, lane, gw); break;
-    case 8: chunk_finalize<DK, CWT, 8>(st, lay, g_lane, scale, lane, gw); break;
+    case 1: chunk_finalize<DK, NF, 1>(vb, lay, g_lane, scale, lane, fw); break;
+    case 2: chunk_finalize<DK, NF, 2>(vb, lay, g_lane, scale, lane, fw); break;
+    case 3: chunk_finalize<DK, NF, 3>(vb, lay, g_lane, scale, lane, fw); break;
+    case 4: chunk_finalize<DK, NF, 4>(vb, lay, g_lane, scale, lane, fw); break;
+    case 5: chunk_finalize<DK, NF, 5>(vb, lay, g_lane, scale, lane, fw); break;
+    case 6: chunk_finalize<DK, NF, 6>(vb, lay, g_lane, scale, lane, fw); break;
+    case 7: chunk_finalize<DK, NF, 7>(vb, lay, g_lane, scale, lane, fw); break;
+    case 8: chunk_finalize<DK, NF, 8>(vb, lay, g_lane, scale, lane, fw); break;
     default: break;
   }
 }
@@ -312,16 +323,22 @@ __device__ __forceinline__ void chunk_sums(const uint8_t* st, const float* su, c
   for (int v = 0; v < 2 * LS; ++v)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[v][c] = 0ull;  // (+0.0f, +0.0f)
+  int off[4];
+  quad_offsets<DK>(rg, c0, off);
+  const float* su_m = su + T0 * DK + 4 * rg;
+  const float* sw_m = sw + T0 * DK + 4 * rg;
+  const uint8_t* st_m = st;
 #pragma unroll 1
-  for (int m = 0; m < DK / 16; ++m) {
-    const int r0 = 16 * m + 4 * rg;
+  for (int m = 0; m < DK / 16; ++m, st_m += kQuadStep, su_m += 16, sw_m += 16) {
     unsigned long long x0[4], x1[4];
-    row_pair_columns(state_quad<DK>(st, r0, c0), state_quad<DK>(st, r0 + 1, c0), x0);
-    row_pair_columns(state_quad<DK>(st, r0 + 2, c0), state_quad<DK>(st, r0 + 3, c0), x1);
+    row_pair_columns(*reinterpret_cast<const uint2*>(st_m + off[0]),
+                     *reinterpret_cast<const uint2*>(st_m + off[1]), x0);
+    row_pair_columns(*reinterpret_cast<const uint2*>(st_m + off[2]),
+                     *reinterpret_cast<const uint2*>(st_m + off[3]), x1);
 #pragma unroll
     for (int t = 0; t < LS; ++t) {
-      const ulonglong2 uq = *reinterpret_cast<const ulonglong2*>(su + (T0 + t) * DK + r0);
-      const ulonglong2 wq = *reinterpret_cast<const ulonglong2*>(sw + (T0 + t) * DK + r0);
+      const ulonglong2 uq = *reinterpret_cast<const ulonglong2*>(su_m + t * DK);
+      const ulonglong2 wq = *reinterpret_cast<const ulonglong2*>(sw_m + t * DK);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         acc[t][c] = fma2(x0[c], uq.x, acc[t][c]);
@@ -361,16 +378,17 @@ __device__ __forceinline__ void chunk_sums(const uint8_t* st, const float* su, c
 }
 
 // One tile with L = LC tokens, for one consumer warp (columns [c0, c0 + 4)
-// of the tile in this lane). `dst` points at row 0, column c0 of the slot's
-// slice; `out_t0` at token 0, column 0 of the tile's output.
+// of the tile in this lane): state tile `st`, vector block `vb`. `dst` points
+// at row 0, column c0 of the slot's slice; `out_t0` at token 0, column 0 of
+// the tile's output.
 template <int DK, int VS, int LC>
-__device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayout& lay, int c0,
-                                              int rg, int lane, uint16_t* dst, uint16_t* out_t0,
-                                              int D_v, uint32_t sum_bar, uint32_t phase) {
-  const float* su = reinterpret_cast<const float*>(st + lay.u);
-  const float* sw = reinterpret_cast<const float*>(st + lay.w);
-  const float* se = reinterpret_cast<const float*>(st + lay.e);
-  const float* sc = reinterpret_cast<const float*>(st + lay.c);
+__device__ __forceinline__ void chunk_consume(const uint8_t* st, const uint8_t* vb,
+                                              const ChunkLayout& lay, int c0, int rg, int lane,
+                                              uint16_t* dst, uint16_t* out_t0, int D_v) {
+  const float* su = reinterpret_cast<const float*>(vb + lay.u);
+  const float* sw = reinterpret_cast<const float*>(vb + lay.w);
+  const float* se = reinterpret_cast<const float*>(vb + lay.e);
+  const float* sc = reinterpret_cast<const float*>(vb + lay.c);
 
   // ---- pass 1: column sums, at most four tokens per sweep of the state
   float ms[LC], ps[LC];
@@ -381,12 +399,11 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayo
                                                                    ps);
 
   // ---- delta (unit lower-triangular solve) and o, for the solved column
-  if (!mbar_wait_bounded(sum_bar, phase)) flag_error(kErrConsumerWait);  // A and B summed
   const int col = c0 + solved_column(rg);
-  const float* sa = reinterpret_cast<const float*>(st + lay.a);
-  const float* sb = reinterpret_cast<const float*>(st + lay.bm);
-  const float* sbeta = reinterpret_cast<const float*>(st + lay.beta);
-  const uint16_t* sv = reinterpret_cast<const uint16_t*>(st + lay.v);
+  const float* sa = reinterpret_cast<const float*>(vb + lay.a);
+  const float* sb = reinterpret_cast<const float*>(vb + lay.bm);
+  const uint16_t* sv = reinterpret_cast<const uint16_t*>(vb + lay.v);
+  const float* sbeta = reinterpret_cast<const float*>(vb + lay.beta);
   float dl[LC];
 #pragma unroll
   for (int t = 0; t < LC; ++t) {
@@ -411,13 +428,21 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayo
     }
 
   // ---- pass 2: S_L = c o S_0 + sum_s e_s delta_s^T, bf16 once, to the slot
+  int off[4];
+  quad_offsets<DK>(rg, c0, off);
+  const uint8_t* st_m = st;
+  const float* sc_m = sc + 4 * rg;
+  const float* se_m = se + 4 * rg;
+  uint16_t* d0 = dst + static_cast<size_t>(4 * rg) * D_v;
+  const size_t d_step = static_cast<size_t>(16) * D_v;
 #pragma unroll 1
-  for (int m = 0; m < DK / 16; ++m) {
-    const int r0 = 16 * m + 4 * rg;
+  for (int m = 0; m < DK / 16; ++m, st_m += kQuadStep, sc_m += 16, se_m += 16, d0 += d_step) {
     unsigned long long n0[4], n1[4];
-    row_pair_columns(state_quad<DK>(st, r0, c0), state_quad<DK>(st, r0 + 1, c0), n0);
-    row_pair_columns(state_quad<DK>(st, r0 + 2, c0), state_quad<DK>(st, r0 + 3, c0), n1);
-    const ulonglong2 cq = *reinterpret_cast<const ulonglong2*>(sc + r0);
+    row_pair_columns(*reinterpret_cast<const uint2*>(st_m + off[0]),
+                     *reinterpret_cast<const uint2*>(st_m + off[1]), n0);
+    row_pair_columns(*reinterpret_cast<const uint2*>(st_m + off[2]),
+                     *reinterpret_cast<const uint2*>(st_m + off[3]), n1);
+    const ulonglong2 cq = *reinterpret_cast<const ulonglong2*>(sc_m);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       n0[c] = mul2(n0[c], cq.x);
@@ -425,7 +450,7 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayo
     }
 #pragma unroll
     for (int s = 0; s < LC; ++s) {
-      const ulonglong2 eq = *reinterpret_cast<const ulonglong2*>(se + s * DK + r0);
+      const ulonglong2 eq = *reinterpret_cast<const ulonglong2*>(se_m + s * DK);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         n0[c] = fma2(eq.x, dd[s][c], n0[c]);
@@ -438,7 +463,6 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayo
       a[c] = upk(n0[c]);
       b[c] = upk(n1[c]);
     }
-    uint16_t* d0 = dst + static_cast<size_t>(r0) * D_v;
     __stcs(reinterpret_cast<uint2*>(d0),
            make_uint2(pack_bf16x2(a[0].x, a[1].x), pack_bf16x2(a[2].x, a[3].x)));
     __stcs(reinterpret_cast<uint2*>(d0 + D_v),
@@ -451,85 +475,113 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const ChunkLayo
 }
 
 template <int DK, int VS>
-__device__ __forceinline__ void chunk_consume_any(int L, const uint8_t* st, const ChunkLayout& lay,
-                                                  int c0, int rg, int lane, uint16_t* dst,
-                                                  uint16_t* out_t0, int D_v, uint32_t sum_bar,
-                                                  uint32_t phase) {
+__device__ __forceinline__ void chunk_consume_any(int L, const uint8_t* st, const uint8_t* vb,
+                                                  const ChunkLayout& lay, int c0, int rg, int lane,
+                                                  uint16_t* dst, uint16_t* out_t0, int D_v) {
   switch (L) {
-    case 1: chunk_consume<DK, VS, 1>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 2: chunk_consume<DK, VS, 2>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 3: chunk_consume<DK, VS, 3>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 4: chunk_consume<DK, VS, 4>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 5: chunk_consume<DK, VS, 5>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 6: chunk_consume<DK, VS, 6>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 7: chunk_consume<DK, VS, 7>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
-    case 8: chunk_consume<DK, VS, 8>(st, lay, c0, rg, lane, dst, out_t0, D_v, sum_bar, phase); break;
+    case 1: chunk_consume<DK, VS, 1>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 2: chunk_consume<DK, VS, 2>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 3: chunk_consume<DK, VS, 3>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 4: chunk_consume<DK, VS, 4>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 5: chunk_consume<DK, VS, 5>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 6: chunk_consume<DK, VS, 6>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 7: chunk_consume<DK, VS, 7>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 8: chunk_consume<DK, VS, 8>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
     default: break;
   }
 }
 
 // ---------------------------------------------------------------- the kernel
 
-// Block: NG groups of VS / 32 consumer warps, then the marker and producer
-// warps; NG = (blockDim.x / 32 - 2) / (VS / 32). Requires n_stages >= NG + 1:
-// tiles are marked ready in order, so a group never waits on a stage two
-// phases ahead of it.
+// Block: NG groups of VS / 32 consumer warps, then kChunkFinalizers finaliser
+// warps, then the producer warp; NG = (blockDim.x / 32 - 1 - kChunkFinalizers)
+// / (VS / 32). Requires n_stages >= NG + 1: tiles are finalised in tile order,
+// so a group never waits on a stage two phases ahead of it.
 template <int DK, int VS, bool GATED>
 __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     decode_chunk_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                         const int n_tiles, const int n_stages) {
   using Shape = ChunkShape<DK, VS>;
   constexpr int CWT = Shape::kWarpsPerTile;
+  constexpr int NF = kChunkFinalizers;
   const int T = p.T;
   const ChunkLayout lay = chunk_layout<DK, VS>(T);
 
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_base = smem_addr(smem_raw);
   uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + n_stages * lay.bytes);
-  const uint32_t raw0 = smem_addr(bars);         // copies landed
-  const uint32_t full0 = raw0 + 8 * n_stages;    // tile ready (in tile order)
-  const uint32_t fin0 = full0 + 8 * n_stages;    // the group's row vectors are written
-  const uint32_t sum0 = fin0 + 8 * n_stages;     // the group's A and B are summed
-  const uint32_t empty0 = sum0 + 8 * n_stages;   // the group is done with the stage
+  uint8_t* vec_base = smem + n_stages * Shape::kStateBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(vec_base + n_stages * lay.bytes);
+  const uint32_t vec0 = smem_addr(bars);        // k, q, gk rows and gate scalars landed
+  const uint32_t sta0 = vec0 + 8 * n_stages;    // state tile landed
+  const uint32_t full0 = sta0 + 8 * n_stages;   // tile finalised (in tile order)
+  const uint32_t empty0 = full0 + 8 * n_stages; // the group is done with the stage
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int producer = static_cast<int>(blockDim.x >> 5) - 1;
-  const int marker = producer - 1;
-  const int n_groups = marker / CWT;
+  const int first_finalizer = producer - NF;
+  const int n_groups = first_finalizer / CWT;
   const int n_slices = p.D_v / VS;
   const int n_mine = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                      static_cast<int>(gridDim.x);
 
   if (tid == 0) {
     for (int i = 0; i < n_stages; ++i) {
-      mbar_init(raw0 + 8 * i, 32);     // one cp.async arrival per producer lane
-      mbar_init(full0 + 8 * i, 1);
-      mbar_init(fin0 + 8 * i, CWT);    // one arrival per warp of the group
-      mbar_init(sum0 + 8 * i, CWT);
-      mbar_init(empty0 + 8 * i, CWT);
+      mbar_init(vec0 + 8 * i, 32);     // one cp.async arrival per producer lane
+      mbar_init(sta0 + 8 * i, 1);      // the producer's lane 0 (+ the TMA bytes)
+      mbar_init(full0 + 8 * i, NF);    // one arrival per finaliser warp
+      mbar_init(empty0 + 8 * i, CWT);  // one arrival per warp of the group
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == marker) {
-    // ================================================================ marker
-    // Tiles become ready in tile order; so a group that waits for tile x
-    // finds the stage's barrier at tile x's phase (tile x - n_stages was
-    // marked before it). Waiting on every tile's copies also means the CTA
-    // never retires with copies in flight.
-    if (lane == 0) {
-      for (int j = 0; j < n_mine; ++j) {
-        const int stage = j % n_stages;
-        if (!mbar_wait_bounded(raw0 + 8 * stage, (j / n_stages) & 1)) flag_error(kErrProducerWait);
-        mbar_arrive(full0 + 8 * stage);
+  if (warp >= first_finalizer && warp < producer) {
+    // ================================================================ finalisers
+    // Every tile in tile order: wait for its vectors (not for the state),
+    // compute the gate and this warp's rows of u, w, e, c and partial sums of
+    // A and B, and mark the tile finalised.
+    const int fw = warp - first_finalizer;
+    for (int j = 0; j < n_mine; ++j) {
+      const int tile = blockIdx.x + j * gridDim.x;
+      const int h = (tile / n_slices) % p.H_v;
+      const int b = tile / (n_slices * p.H_v);
+      const int stage = j % n_stages;
+      uint8_t* vb = vec_base + stage * lay.bytes;
+      if (!mbar_wait_bounded(vec0 + 8 * stage, (j / n_stages) & 1)) flag_error(kErrProducerWait);
+      int L = reinterpret_cast<const int*>(vb + lay.meta)[0];
+      L = L < 0 ? 0 : (L > T ? T : L);
+      if (L > 0) {
+        float gt = 0.0f;
+        if (lane < L) {  // the gate of token `lane`
+          const uint32_t* rawv = reinterpret_cast<const uint32_t*>(vb + lay.raw);
+          float bt;
+          if constexpr (GATED) {
+            const size_t ai = (static_cast<size_t>(b) * T + lane) * p.H_v + h;
+            const float dtb = __uint_as_float(rawv[16]);
+            const float dsc = __uint_as_float(rawv[17]);
+            gt = dsc * softplus_f32(bf16_in_word(rawv[lane], p.gate_a + ai) + dtb);  // g
+            bt = sigmoid_f32(bf16_in_word(rawv[8 + lane], p.gate_b + ai));          // beta
+          } else {
+            const size_t gi = (static_cast<size_t>(b) * p.H_v + h) * T + lane;
+            gt = __uint_as_float(rawv[lane]);
+            bt = bf16_in_word(rawv[8 + lane], p.beta + gi);
+          }
+          if (fw == 0) reinterpret_cast<float*>(vb + lay.beta)[lane] = bt;
+        }
+        chunk_finalize_any<DK, NF>(L, vb, lay, gt, p.scale, lane, fw);
       }
+      named_barrier(1, 32 * NF);  // every finaliser takes the same path: no early exits
+      if (L > 0) chunk_sum_parts<NF>(vb, lay, L, lane, fw);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full0 + 8 * stage);
     }
+    // (the consumers wait for every state tile, so no copy outlives the CTA)
     return;
   }
+
   if (warp == producer) {
     // ================================================================ producer
     bool failed = false;
@@ -563,8 +615,9 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       if (s < 0 || s >= p.pool_size) L = 0;
       const int stage = j % n_stages;
       const uint32_t phase = (j / n_stages) & 1;
-      uint8_t* st = smem + stage * lay.bytes;
-      const uint32_t rawb = raw0 + 8 * stage;
+      uint8_t* vb = vec_base + stage * lay.bytes;
+      const uint32_t vbar = vec0 + 8 * stage;
+      const uint32_t sbar = sta0 + 8 * stage;
       if (lane == 0 && !failed) {
         if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1)) {
           failed = true;
@@ -573,31 +626,34 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        int* meta = reinterpret_cast<int*>(st + lay.meta);
+        int* meta = reinterpret_cast<int*>(vb + lay.meta);
         meta[0] = L;
         meta[1] = s;
         if (L > 0) {
-          mbar_expect_tx(rawb, Shape::kStateBytes + L * (VS * 2 + DK * 8));
           // the L valid tokens' rows are contiguous in HBM: one copy each
-          const int col0 = slice * VS;
+          mbar_expect_tx(vbar, L * (DK * 8 + VS * 2));
+          mbar_expect_tx(sbar, Shape::kStateBytes);
           const size_t qk_off = (static_cast<size_t>(b) * p.H_qk + h / p.group) * T * DK;
           const size_t gk_off = (static_cast<size_t>(b) * p.H_v + h) * T * DK;
-          const uint16_t* vsrc = p.value + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + col0;
-          tma_load_3d(smem_addr(st), &pool_map, 0, (s * p.H_v + h) * DK, col0 / 64, rawb);
-          bulk_load(smem_addr(st + lay.k), p.key + qk_off, L * DK * 2, rawb);
-          bulk_load(smem_addr(st + lay.q), p.query + qk_off, L * DK * 2, rawb);
-          bulk_load(smem_addr(st + lay.u), p.gk + gk_off, L * DK * 4, rawb);
+          bulk_load(smem_addr(vb + lay.k), p.key + qk_off, L * DK * 2, vbar);
+          bulk_load(smem_addr(vb + lay.q), p.query + qk_off, L * DK * 2, vbar);
+          bulk_load(smem_addr(vb + lay.u), p.gk + gk_off, L * DK * 4, vbar);
+          const uint16_t* vsrc =
+              p.value + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + slice * VS;
           if (VS == p.D_v) {
-            bulk_load(smem_addr(st + lay.v), vsrc, L * VS * 2, rawb);
+            bulk_load(smem_addr(vb + lay.v), vsrc, L * VS * 2, vbar);
           } else {
             for (int t = 0; t < L; ++t)
-              bulk_load(smem_addr(st + lay.v + t * VS * 2), vsrc + static_cast<size_t>(t) * p.D_v,
-                        VS * 2, rawb);
+              bulk_load(smem_addr(vb + lay.v + t * VS * 2), vsrc + static_cast<size_t>(t) * p.D_v,
+                        VS * 2, vbar);
           }
+          tma_load_3d(smem_addr(smem + stage * Shape::kStateBytes), &pool_map, 0,
+                      (s * p.H_v + h) * DK, slice * VS / 64, sbar);
         }
+        mbar_arrive(sbar);
       }
       // gate scalars: lane t fetches token t's pair; lane 31 the per-head values
-      uint32_t* rawv = reinterpret_cast<uint32_t*>(st + lay.raw);
+      uint32_t* rawv = reinterpret_cast<uint32_t*>(vb + lay.raw);
       if (lane < L) {
         if constexpr (GATED) {
           const size_t ai = (static_cast<size_t>(b) * T + lane) * p.H_v + h;
@@ -615,7 +671,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
           cp_async_4(smem_addr(rawv + 17), p.decay_scale + h);
         }
       }
-      cp_async_arrive_noinc(rawb);
+      cp_async_arrive_noinc(vbar);
     }
     return;
   }
@@ -626,6 +682,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
   const int gw = warp % CWT;
   const int rg = lane >> 3;
   const int c0 = gw * kChunkWarpCols + (lane & 7) * 4;  // first tile column of this lane
+  const int col = c0 + solved_column(rg);               // the column this lane solves
   for (int it = group; it < n_mine; it += n_groups) {
     const int tile = blockIdx.x + it * gridDim.x;
     const int slice = tile % n_slices;
@@ -633,59 +690,30 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     const int b = tile / (n_slices * p.H_v);
     const int stage = it % n_stages;
     const uint32_t phase = (it / n_stages) & 1;
-    uint8_t* st = smem + stage * lay.bytes;
+    const uint8_t* st = smem + stage * Shape::kStateBytes;
+    const uint8_t* vb = vec_base + stage * lay.bytes;
 
-    const bool ok_self = mbar_wait_bounded(full0 + 8 * stage, phase);
+    // finalised (in tile order), then the state tile itself: it was issued
+    // before the tile was finalised, so its barrier is at this tile's phase
+    bool ok_self = mbar_wait_bounded(full0 + 8 * stage, phase);
+    ok_self = mbar_wait_bounded(sta0 + 8 * stage, phase) && ok_self;
     const bool ok = __all_sync(0xffffffffu, ok_self);
     if (!ok_self) flag_error(kErrConsumerWait);
-    const int* meta = reinterpret_cast<const int*>(st + lay.meta);
+    const int* meta = reinterpret_cast<const int*>(vb + lay.meta);
     int L = ok ? meta[0] : 0;
     L = L < 0 ? 0 : (L > T ? T : L);
     const int s = meta[1];
     if (s < 0 || s >= p.pool_size) L = 0;
 
     // out[b, h, t, slice * VS + column]; padded tokens get +0.0
-    uint16_t* out_t0 = p.out + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + slice * VS;
-    const int col = c0 + solved_column(rg);
+    const size_t bh = static_cast<size_t>(b) * p.H_v + h;
+    uint16_t* out_t0 = p.out + bh * T * p.D_v + slice * VS;
     for (int t = L; t < T; ++t) out_t0[static_cast<size_t>(t) * p.D_v + col] = 0;
 
     if (L > 0) {
-      // ---- gate (lane t: token t), then this warp's rows of the finalise step
-      float gt = 0.0f;
-      if (lane < L) {
-        const uint32_t* rawv = reinterpret_cast<const uint32_t*>(st + lay.raw);
-        float bt;
-        if constexpr (GATED) {
-          const size_t ai = (static_cast<size_t>(b) * T + lane) * p.H_v + h;
-          const float dtb = __uint_as_float(rawv[16]);
-          const float dsc = __uint_as_float(rawv[17]);
-          gt = dsc * softplus_f32(bf16_in_word(rawv[lane], p.gate_a + ai) + dtb);  // g
-          bt = sigmoid_f32(bf16_in_word(rawv[8 + lane], p.gate_b + ai));          // beta
-        } else {
-          const size_t gi = (static_cast<size_t>(b) * p.H_v + h) * T + lane;
-          gt = __uint_as_float(rawv[lane]);
-          bt = bf16_in_word(rawv[8 + lane], p.beta + gi);
-        }
-        if (gw == 0) reinterpret_cast<float*>(st + lay.beta)[lane] = bt;
-      }
-      chunk_finalize_any<DK, CWT>(L, st, lay, gt, p.scale, lane, gw);
-    }
-    // The group meets twice: once the row vectors and partial sums are
-    // written, and once A and B are summed (waited for only after pass 1).
-    // Every warp arrives on both, so the phases stay in step.
-    __syncwarp();
-    if (lane == 0) mbar_arrive(fin0 + 8 * stage);
-    if (L > 0) {
-      if (!mbar_wait_bounded(fin0 + 8 * stage, phase)) flag_error(kErrConsumerWait);
-      chunk_sum_parts<CWT>(st, lay, L, lane, gw);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sum0 + 8 * stage);
-    if (L > 0) {
       uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
                       slice * VS + c0;
-      chunk_consume_any<DK, VS>(L, st, lay, c0, rg, lane, dst, out_t0, p.D_v, sum0 + 8 * stage,
-                                phase);
+      chunk_consume_any<DK, VS>(L, st, vb, lay, c0, rg, lane, dst, out_t0, p.D_v);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * stage);

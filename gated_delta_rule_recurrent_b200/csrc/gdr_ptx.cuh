@@ -64,10 +64,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase of parity `parity` to complete, for at most
 // kWaitLimitCycles. Returns false when the budget ran out.
+// As mbar_try_wait, but the thread may stay suspended in the instruction for
+// up to `hint_ns` nanoseconds while the phase is incomplete (it resumes as
+// soon as the phase completes), so a waiting warp takes few issue slots.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_suspend(bar, parity, kWaitSuspendNs)) {
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
   return true;
