@@ -42,6 +42,7 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 DEFAULT_WORKLOAD = 4
 KERNEL_SOURCE_FILES = ("gated_delta_rule_recurrent_b200/csrc/gdr_decode.cuh",
+                       "gated_delta_rule_recurrent_b200/csrc/gdr_ptx.cuh",
                        "gated_delta_rule_recurrent_b200/csrc/gdr_decode_tma.cuh",
                        "gated_delta_rule_recurrent_b200/csrc/gdr_api.cu")
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gated_B512_H64_64x512_dram.txt")

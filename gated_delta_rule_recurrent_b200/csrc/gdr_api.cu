@@ -129,7 +129,7 @@ struct LaunchConfig {
   int ctas_per_sm = 0;
 };
 
-template <int DK, int VS, int R, bool GATED, bool ONE>
+template <int DK, int VS, int R, bool GATED>
 int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
   using Shape = gdr::TmaShape<DK, VS, R>;
   static LaunchConfig cache[kMaxDevices][gdr::kMaxT + 1];
@@ -138,7 +138,7 @@ int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
     *out = cache[dev][T];
     return GDR_OK;
   }
-  auto kernel = gdr::decode_tma_kernel<DK, VS, R, GATED, ONE>;
+  auto kernel = gdr::decode_tma_kernel<DK, VS, R, GATED>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          props.smem_optin);
   // All of the unified L1/shared storage as shared memory, so that the CTAs
@@ -157,12 +157,12 @@ int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
   ctas = ctas < 1 ? 1 : (ctas > 4 ? 4 : ctas);
   LaunchConfig c;
   for (; ctas >= 1; --ctas) {
-    const int stage_bytes = gdr::stage_layout<DK, VS, R, ONE>(T).bytes;
+    const int stage_bytes = gdr::stage_layout<DK, VS, R>(T).bytes;
     const int budget = props.smem_per_sm / ctas - 1024;
-    int n = (budget - 1024 - gdr::cta_extra_bytes<DK, VS, R, ONE>(kMaxStages)) / stage_bytes;
+    int n = (budget - 1024 - gdr::cta_extra_bytes(kMaxStages)) / stage_bytes;
     n = n > kMaxStages ? kMaxStages : n;
     if (n < gdr::kMinStages) n = gdr::kMinStages;
-    const int smem = gdr::tma_smem_bytes<DK, VS, R, ONE>(T, n);
+    const int smem = gdr::tma_smem_bytes<DK, VS, R>(T, n);
     if (smem > props.smem_optin) continue;
     // A persistent grid must be co-resident: trust the occupancy calculator.
     int resident = 0;
@@ -182,7 +182,7 @@ int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
   return GDR_OK;
 }
 
-template <int DK, int VS, int R, bool GATED, bool ONE>
+template <int DK, int VS, int R, bool GATED>
 int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   using Shape = gdr::TmaShape<DK, VS, R>;
   int dev = 0;
@@ -192,7 +192,7 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   LaunchConfig cfg;
-  rc = launch_config<DK, VS, R, GATED, ONE>(dev, p.T, props, &cfg);
+  rc = launch_config<DK, VS, R, GATED>(dev, p.T, props, &cfg);
   if (rc != GDR_OK) return rc;
   const int n_stages = cfg.n_stages;
   const int smem = cfg.smem;
@@ -205,7 +205,7 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   const int n_tiles = p.B * p.H_v * (p.D_v / VS);
   const int max_ctas = ctas_per_sm * props.sms;
   const int grid = n_tiles < max_ctas ? n_tiles : max_ctas;
-  gdr::decode_tma_kernel<DK, VS, R, GATED, ONE><<<grid, Shape::kThreads, smem, stream>>>(map, p, n_tiles,
+  gdr::decode_tma_kernel<DK, VS, R, GATED><<<grid, Shape::kThreads, smem, stream>>>(map, p, n_tiles,
                                                                                  n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
@@ -307,13 +307,13 @@ struct SliceKernel {
 // the chunked kernel (64 columns per consumer warp).
 template <bool GATED>
 const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
-  static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED, true>},
-                                        {256, launch_tma<64, 256, 8, GATED, true>},
-                                        {128, launch_tma<64, 128, 8, GATED, true>},
-                                        {64, launch_tma<64, 64, 8, GATED, true>}};
-  static const SliceKernel k128_one[] = {{256, launch_tma<128, 256, 16, GATED, true>},
-                                         {128, launch_tma<128, 128, 16, GATED, true>},
-                                         {64, launch_tma<128, 64, 16, GATED, true>}};
+  static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED>},
+                                        {256, launch_tma<64, 256, 8, GATED>},
+                                        {128, launch_tma<64, 128, 8, GATED>},
+                                        {64, launch_tma<64, 64, 8, GATED>}};
+  static const SliceKernel k128_one[] = {{256, launch_tma<128, 256, 16, GATED>},
+                                         {128, launch_tma<128, 128, 16, GATED>},
+                                         {64, launch_tma<128, 64, 16, GATED>}};
   static const SliceKernel k64_many[] = {{128, launch_chunk<64, 128, GATED>},
                                          {64, launch_chunk<64, 64, GATED>}};
   static const SliceKernel k128_many[] = {{128, launch_chunk<128, 128, GATED>},

@@ -72,8 +72,19 @@ namespace gdr {
 
 constexpr int kChunkWarpCols = 32;      // columns per consumer warp: 8 lanes x 4
 constexpr int kChunkFinalizers = 2;     // warps that turn landed tiles into row vectors
-constexpr int kChunkMaxThreads = 480;   // 12 consumer warps, the finalisers and the producer
-constexpr int kChunkMaxSubTokens = 4;   // tokens per pass-1 sweep
+#ifndef GDR_CHUNK_MAX_THREADS
+#define GDR_CHUNK_MAX_THREADS 352
+#endif
+// Block size cap: consumer groups, the finalisers and the producer. It also
+// caps the registers ptxas may give a thread (up to 384 threads: 168; 480:
+// 128). Two consumer groups with 168 registers run faster than three with
+// 128: with fewer registers the shared-memory loads cannot run ahead of
+// their uses.
+constexpr int kChunkMaxThreads = GDR_CHUNK_MAX_THREADS;
+#ifndef GDR_CHUNK_SWEEP_TOKENS
+#define GDR_CHUNK_SWEEP_TOKENS 4
+#endif
+constexpr int kChunkMaxSubTokens = GDR_CHUNK_SWEEP_TOKENS;  // tokens per pass-1 sweep
 
 template <int DK, int VS>
 struct ChunkShape {

@@ -1,4 +1,6 @@
-// Persistent, warp-specialised decode kernel for sm_100a.
+// Persistent, warp-specialised single-token decode kernel for sm_100a (calls
+// with T = 1, the common decode step; calls with T > 1 go to the kernel in
+// gdr_decode_chunk.cuh).
 //
 // Arithmetic: the four steps of "lite_boost.ops.recurrent_gated_delta_rule"
 // (MindSpore Lite API page, section 算法流程) and, when GATED, the gate of
@@ -8,26 +10,27 @@
 // state: all D_k rows x VS bf16 columns of slot ssm_state_indices[b]; with
 // VS = D_v it is the slot's whole contiguous head state. Each CTA walks tiles
 // tile = blockIdx.x, + gridDim.x, ... through a ring of shared-memory stages,
-// with three roles:
+// with two roles:
 //
 //   producer warp - starts the asynchronous copies of a tile (one TMA box for
-//           the state; 1-D bulk copies of the value rows and of the k, q and
-//           gk rows of the valid tokens; 4-byte cp.async copies of the
-//           per-token gate scalars) and, kLookahead tiles later, once they
-//           have landed ("raw" barrier), turns them into what the consumers
-//           use: exp(g + gk) per row (written over gk), k.(q*scale) and beta
-//           per token ("full" barrier). No lane waits on global-memory latency.
-//   consumer warps - each owns ALL D_k rows of a band of 32 columns; lane
-//           (row lane 0..7, column lane 0..3) holds D_k/8 rows x 8 columns in
-//           fp32 registers for all valid tokens. Every reduction over D_k is a
-//           warp shuffle, so consumer warps never synchronise with each other
-//           and drift apart freely. Per token: decay in place; the column sums
-//           kv_mem = S^T k and p = S^T q together; a reduce-scatter over the
-//           row lanes; delta; output o = scale * p + delta * (k.q*scale),
-//           which is step 4's S_new^T (q*scale) with the sums reordered;
-//           rank-1 update. A warp gives the stage back ("empty" barrier) as
-//           soon as it has read what it needs, and then streams its rows of the
-//           new state to the pool from registers with 16-byte stores.
+//           the state, 128-byte swizzled; 1-D bulk copies of the value row
+//           and of the k, q and gk rows; 4-byte cp.async copies of the gate
+//           scalars) and, kLookahead tiles later, once they have landed
+//           ("raw" barrier), turns them into what the consumers use: per row
+//           the float4 {d k, d q*scale, d, k} with d = exp(g + gk), in owner
+//           order, and per token k.(q*scale) and beta ("full" barrier). No
+//           lane waits on global-memory latency.
+//   consumer warps - each owns ALL D_k rows of a band of columns; lane (row
+//           lane, column lane) holds R rows x 8 columns. Every reduction over
+//           D_k is a warp shuffle, so consumer warps never synchronise with
+//           each other and drift apart freely. The decay is folded into the
+//           row vectors: kv_mem = S^T (d k) and p = S^T (d q*scale) in one
+//           read of the bf16 rows; a reduce-scatter over the row lanes; delta;
+//           o = p + delta * (k.q*scale), which is step 4's S_new^T (q*scale)
+//           with the sums reordered; then a second read of the rows gives
+//           S_new = d S + k delta^T, rounded to bf16 once and stored straight
+//           to the slot with 16-byte streaming stores. A warp gives the stage
+//           back ("empty" barrier) when it has read what it needs.
 //
 // HBM sees one bulk read and one write of every touched state tile, and a
 // stage is held only while its tile is loaded and computed.
@@ -107,9 +110,9 @@ struct StageLayout {
   int v, k, q, gk, rv, raw, beta, kq, meta, bytes;
 };
 
-// ONE (single-token calls): the producer also writes float4 row vectors
-// {d k, d q_s, d, k}; multi-token calls use the compact form, d written over gk.
-template <int DK, int VS, int R, bool ONE>
+// The producer turns the k, q and gk rows into float4 row vectors
+// {d k, d q_s, d, k} in owner order (see owner_slot).
+template <int DK, int VS, int R>
 __host__ __device__ inline StageLayout stage_layout(int T) {
   StageLayout s;
   s.v = TmaShape<DK, VS, R>::kStateBytes;  // bf16 [T][VS]   value rows of the slice
@@ -118,9 +121,9 @@ __host__ __device__ inline StageLayout stage_layout(int T) {
   constexpr int TS = TmaShape<DK, VS, R>::kTokStride;
   s.k = s.v + T * VS * 2;               // bf16 [T][TS]   key rows
   s.q = s.k + T * TS * 2;               // bf16 [T][TS]   query rows
-  s.gk = s.q + T * TS * 2;              // fp32 [T][TS]   gk rows (multi-token: then d = exp(g + gk))
-  s.rv = s.gk + T * TS * 4;             // fp32x4 [T][TS] {d*k, d*q*scale, d, k} (single-token only)
-  s.raw = s.rv + (ONE ? T * TS * 16 : 0);  // u32 [2][8]  gate scalar words
+  s.gk = s.q + T * TS * 2;              // fp32 [T][TS]   gk rows
+  s.rv = s.gk + T * TS * 4;             // fp32x4 [T][TS] {d*k, d*q*scale, d, k}
+  s.raw = s.rv + T * TS * 16;           // u32 [2][8]  gate scalar words
   s.beta = s.raw + 64;                  // fp32 [8]
   s.kq = s.beta + 32;                   // fp32 [8]       k . (q * scale)
   s.meta = s.kq + 32;                   // int32 [4]      length, slot
@@ -129,22 +132,17 @@ __host__ __device__ inline StageLayout stage_layout(int T) {
 }
 
 // CTA-level area after the stages: three mbarriers per stage.
-template <int DK, int VS, int R, bool ONE>
-__host__ __device__ inline int cta_extra_bytes(int n_stages) {
-  return 3 * n_stages * 8;
-}
+__host__ __device__ inline int cta_extra_bytes(int n_stages) { return 3 * n_stages * 8; }
 
-template <int DK, int VS, int R, bool ONE>
+template <int DK, int VS, int R>
 __host__ __device__ inline int tma_smem_bytes(int T, int n_stages) {
-  return 1024 /* alignment slack */ + n_stages * stage_layout<DK, VS, R, ONE>(T).bytes +
-         cta_extra_bytes<DK, VS, R, ONE>(n_stages);
+  return 1024 /* alignment slack */ + n_stages * stage_layout<DK, VS, R>(T).bytes +
+         cta_extra_bytes(n_stages);
 }
 
 // ---------------------------------------------------------------- the kernel
 
-// ONE: the call has a single token (T = 1), the common decode case; the
-// consumers then keep only bf16 state words between the two passes.
-template <int DK, int VS, int RR, bool GATED, bool ONE>
+template <int DK, int VS, int RR, bool GATED>
 __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     decode_tma_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                       const int n_tiles, const int n_stages) {
@@ -157,7 +155,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
   constexpr int NV = 16 / RL;  // reduced values per lane after the reduce-scatter: 4, 2 or 1
   constexpr int TS = Shape::kTokStride;
   const int T = p.T;
-  const StageLayout lay = stage_layout<DK, VS, RR, ONE>(T);
+  const StageLayout lay = stage_layout<DK, VS, RR>(T);
 
   // Stages start on a 1024-byte boundary of the shared window. The offset is
   // added to the __shared__ array itself so every access stays a shared-memory
@@ -289,8 +287,6 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         float4* srv = reinterpret_cast<float4*>(st + lay.rv);
         const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);
         const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
-        uint16_t* skw = reinterpret_cast<uint16_t*>(st + lay.k);
-        uint16_t* sqw = reinterpret_cast<uint16_t*>(st + lay.q);
         float dtb = 0.0f, dsc = 0.0f;
         if constexpr (GATED) {
           if (L > 0) {
@@ -313,33 +309,21 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
             gt = __uint_as_float(rawv[t]);
             bt = bf16_in_word(rawv[8 + t], p.beta + gi);
           }
-          // Row vectors go to owner order (see owner_slot): read every row of
-          // this token first, then write, so the in-place permutation of the
-          // multi-token arrays is safe.
+          // Row vectors go to owner order (see owner_slot).
           float kq = 0.0f;
           float dv[E], kv[E], qv[E];
-          uint16_t kb[E], qb[E];
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const int i = lane + 32 * e;
             dv[e] = expf(gt + sgk[t * TS + i]);  // exp(g) * exp(gk) as one exponential
-            kb[e] = sk[t * TS + i];
-            qb[e] = sq[t * TS + i];
-            kv[e] = bf16_bits_to_f32(kb[e]);
-            qv[e] = bf16_bits_to_f32(qb[e]) * p.scale;
+            kv[e] = bf16_bits_to_f32(sk[t * TS + i]);
+            qv[e] = bf16_bits_to_f32(sq[t * TS + i]) * p.scale;
             kq = fmaf(kv[e], qv[e], kq);
           }
-          __syncwarp();
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             const int o = t * TS + owner_slot<RL, R>(lane + 32 * e);
-            if constexpr (ONE) {
-              srv[o] = make_float4(dv[e] * kv[e], dv[e] * qv[e], dv[e], kv[e]);
-            } else {
-              sgk[o] = dv[e];
-              skw[o] = kb[e];
-              sqw[o] = qb[e];
-            }
+            srv[o] = make_float4(dv[e] * kv[e], dv[e] * qv[e], dv[e], kv[e]);
           }
           kq = warp_sum(kq);
           __syncwarp();
@@ -393,7 +377,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     const int* meta = reinterpret_cast<const int*>(st + lay.meta);
     int L = ok ? meta[0] : 0;  // one load for the whole warp: every lane sees one value
     L = L < 0 ? 0 : (L > T ? T : L);
-    if constexpr (ONE) L = L > 1 ? 1 : L;
+    L = L > 1 ? 1 : L;  // single-token calls
     const int s = meta[1];
     if (s < 0 || s >= p.pool_size) L = 0;
 
@@ -407,29 +391,13 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
           make_uint4(0u, 0u, 0u, 0u);
     }
 
-    // Multi-token calls keep the state in fp32 registers across tokens:
-    // S2[r][c] holds columns c0 + 2c, c0 + 2c + 1 of row i0 + r as a packed
-    // pair. A single-token call keeps no state in registers: it reads its rows
-    // from the stage once for the column sums and once more for the update,
-    // and streams each new row to the pool straight from the update.
-    unsigned long long S2[ONE ? 1 : R][4];
+    // No state is kept in registers: a warp reads its rows from the stage
+    // once for the column sums and once more for the update, and streams each
+    // new row to the pool straight from the update.
     uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
                     slice * VS + c0;  // + row * D_v
     if (L > 0) {
-      if constexpr (!ONE) {
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint4 w = *reinterpret_cast<const uint4*>(st + swz_offset<DK>(r * RL + rp, c0));
-          S2[r][0] = pk(bf16_lo(w.x), bf16_hi(w.x));
-          S2[r][1] = pk(bf16_lo(w.y), bf16_hi(w.y));
-          S2[r][2] = pk(bf16_lo(w.z), bf16_hi(w.z));
-          S2[r][3] = pk(bf16_lo(w.w), bf16_hi(w.w));
-        }
-      }
-      const float4* srv = reinterpret_cast<const float4*>(st + lay.rv);  // single-token
-      const uint16_t* sk = reinterpret_cast<const uint16_t*>(st + lay.k);  // multi-token
-      const uint16_t* sq = reinterpret_cast<const uint16_t*>(st + lay.q);
-      const float* sd = reinterpret_cast<const float*>(st + lay.gk);
+      const float4* srv = reinterpret_cast<const float4*>(st + lay.rv);
       const float* sbeta = reinterpret_cast<const float*>(st + lay.beta);
       const float* skq = reinterpret_cast<const float*>(st + lay.kq);
       const uint16_t* sv = reinterpret_cast<const uint16_t*>(st + lay.v);
@@ -440,9 +408,9 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         unsigned long long m2[4], p2[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) m2[c] = p2[c] = 0ull;  // (+0.0f, +0.0f)
-        // (single-token rows are re-read from shared memory, so their loop
-        // need not be unrolled: unrolling it fully only raises register use)
-        if constexpr (ONE) {
+        // (the rows are re-read from shared memory, so the loop need not be
+        // unrolled: unrolling it fully only raises register use)
+        {
 #pragma unroll 2
           for (int r = 0; r < R; ++r) {
             const float2 rv0 = reinterpret_cast<const float2*>(srv + t * TS + i0 + r)[0];
@@ -455,27 +423,6 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
               const unsigned long long sr = pk(bf16_lo(wv[c]), bf16_hi(wv[c]));
               m2[c] = fma2(sr, dk2, m2[c]);  // steps 1-2: kv_mem partial
               p2[c] = fma2(sr, dq2, p2[c]);  // S_dec^T q_s partial
-            }
-          }
-        } else {
-#pragma unroll
-          for (int r4 = 0; r4 < R; r4 += 4) {
-            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * TS + i0 + r4);
-            const uint2 qw = *reinterpret_cast<const uint2*>(sq + t * TS + i0 + r4);
-            const float4 dw = *reinterpret_cast<const float4*>(sd + t * TS + i0 + r4);
-            const float kr[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
-            const float qr[4] = {bf16_lo(qw.x), bf16_hi(qw.x), bf16_lo(qw.y), bf16_hi(qw.y)};
-            const float dr[4] = {dw.x, dw.y, dw.z, dw.w};
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-              const float dk = dr[rr] * kr[rr], dq = dr[rr] * qr[rr];
-              const unsigned long long dk2 = pk(dk, dk);
-              const unsigned long long dq2 = pk(dq, dq);
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                m2[c] = fma2(S2[r4 + rr][c], dk2, m2[c]);  // steps 1-2: kv_mem partial
-                p2[c] = fma2(S2[r4 + rr][c], dq2, p2[c]);  // S_dec^T q partial (unscaled)
-              }
             }
           }
         }
@@ -549,19 +496,17 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
           if (b4) dlt[c] = other;
         }
         if (b4) {
-          const float kq = skq[t];
-          // single-token p already carries the query scale; multi-token p does not
-          const float ps = ONE ? 1.0f : p.scale;
+          const float kq = skq[t];  // p already carries the query scale
           uint16_t* dst = out_band + static_cast<size_t>(t) * p.D_v + cred;
           if constexpr (NV == 4) {
             *reinterpret_cast<uint2*>(dst) =
-                make_uint2(pack_bf16x2(fmaf(dlt[0], kq, red[0] * ps), fmaf(dlt[1], kq, red[1] * ps)),
-                           pack_bf16x2(fmaf(dlt[2], kq, red[2] * ps), fmaf(dlt[3], kq, red[3] * ps)));  // step 4
+                make_uint2(pack_bf16x2(fmaf(dlt[0], kq, red[0]), fmaf(dlt[1], kq, red[1])),
+                           pack_bf16x2(fmaf(dlt[2], kq, red[2]), fmaf(dlt[3], kq, red[3])));  // step 4
           } else if constexpr (NV == 2) {
             *reinterpret_cast<uint32_t*>(dst) =
-                pack_bf16x2(fmaf(dlt[0], kq, red[0] * ps), fmaf(dlt[1], kq, red[1] * ps));  // step 4
+                pack_bf16x2(fmaf(dlt[0], kq, red[0]), fmaf(dlt[1], kq, red[1]));  // step 4
           } else {
-            *dst = f32_to_bf16_bits(fmaf(dlt[0], kq, red[0] * ps));  // step 4
+            *dst = f32_to_bf16_bits(fmaf(dlt[0], kq, red[0]));  // step 4
           }
         }
         // every lane gathers delta of its own 8 columns from the kv_mem lanes
@@ -576,7 +521,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) dl2[c] = pk(dl[2 * c], dl[2 * c + 1]);
         // steps 1 and 3: S_new = d S + k delta^T
-        if constexpr (ONE) {
+        {
 #pragma unroll 2
           for (int r = 0; r < R; ++r) {
             const float2 rv1 = reinterpret_cast<const float2*>(srv + t * TS + i0 + r)[1];
@@ -592,45 +537,12 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
                    make_uint4(pack_bf16x2(n0.x, n0.y), pack_bf16x2(n1.x, n1.y),
                               pack_bf16x2(n2.x, n2.y), pack_bf16x2(n3.x, n3.y)));
           }
-        } else {
-#pragma unroll
-          for (int r4 = 0; r4 < R; r4 += 4) {
-            const uint2 kw = *reinterpret_cast<const uint2*>(sk + t * TS + i0 + r4);
-            const float4 dw = *reinterpret_cast<const float4*>(sd + t * TS + i0 + r4);
-            const float kr[4] = {bf16_lo(kw.x), bf16_hi(kw.x), bf16_lo(kw.y), bf16_hi(kw.y)};
-            const float dr[4] = {dw.x, dw.y, dw.z, dw.w};
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-              const unsigned long long d2 = pk(dr[rr], dr[rr]);
-              const unsigned long long k2 = pk(kr[rr], kr[rr]);
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                S2[r4 + rr][c] = fma2(S2[r4 + rr][c], d2, mul2(k2, dl2[c]));
-            }
-          }
         }
       }
     }
     // This warp has read everything it needs from the stage: give it back.
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * stage);
-
-    if (!ONE && L > 0) {
-      // The new state, bf16 round-to-nearest-even once per call, streamed from
-      // registers to the slot with 16-byte stores.
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        uint4 o;
-        {
-          float2 v;
-          v = upk(S2[r][0]); o.x = pack_bf16x2(v.x, v.y);
-          v = upk(S2[r][1]); o.y = pack_bf16x2(v.x, v.y);
-          v = upk(S2[r][2]); o.z = pack_bf16x2(v.x, v.y);
-          v = upk(S2[r][3]); o.w = pack_bf16x2(v.x, v.y);
-        }
-        __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r * RL + rp) * p.D_v), o);
-      }
-    }
   }
 }
 

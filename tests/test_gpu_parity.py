@@ -91,6 +91,30 @@ def test_every_token_count(T):
     _roundtrip(workloads.make_inputs(w), False)
 
 
+@pytest.mark.parametrize("regime", ["vanishing", "none", "mixed"])
+def test_decay_regimes_multi_token(regime):
+    """Multi-token calls regroup the recurrence around running products of the
+    per-token decays. "vanishing": g = -30 and gk = -5, so the products fall
+    below the fp32 range within a few tokens (the state forgets, nothing may
+    overflow or turn NaN); "none": g = gk = 0 with beta near 1 (the pure delta
+    rule, where the regrouped sums cancel the most); "mixed": alternating
+    strong and weak decay per token and per row."""
+    w = workloads.WORKLOADS[3].replace(name=f"decay_{regime}", B=12, pool=16, seed=321)
+    x = workloads.make_inputs(w)
+    if regime == "vanishing":
+        x["g"][:] = -30.0
+        x["gk"][:] = -5.0
+    elif regime == "none":
+        x["g"][:] = 0.0
+        x["gk"][:] = 0.0
+        x["beta"][:] = 0.99609375  # bf16 just below 1
+    else:
+        x["g"][:, :, 0::2] = -12.0
+        x["g"][:, :, 1::2] = -0.01
+        x["gk"][..., 0::3] = -8.0
+    _roundtrip(x, False)
+
+
 @pytest.mark.parametrize("gated", [False, True])
 def test_edge_lengths_and_slots(gated):
     w = workloads.WORKLOADS[0].replace(name="edges", B=8, H_qk=2, H_v=4, T=4, D_k=128,
