@@ -459,6 +459,94 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_gate(args):
+    """The standalone LinearAttentionGate op on one GPU: one JSON line of its own
+    (elements per second, and achieved HBM GB/s against the measured copy peak)."""
+    import gated_delta_rule_recurrent_b200 as gdr
+    from gated_delta_rule_recurrent_b200 import binding
+
+    binding.lib()  # fail loudly now if the library is missing
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dtype = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[args.gate_dtype]
+    shape = tuple(int(v) for v in args.gate_shape.split("x"))
+    x = workloads.make_gate_inputs(shape, dtype, seed=2024)
+    xd = {k: v.to(dev) for k, v in x.items()}
+    decay = torch.empty_like(xd["a"])
+    beta = torch.empty_like(xd["a"])
+    n = xd["a"].numel()
+    esize = xd["a"].element_size()
+    step_bytes = 4 * n * esize + 2 * 4 * shape[-1]  # a, b in; decay, beta out; per-head vectors
+
+    def step():
+        gdr.linear_attention_gate(xd["a"], xd["dt_bias"], xd["decay_scale"], b=xd["b"],
+                                  decay=decay, beta=beta)
+
+    sampler = ClockSampler(0)
+    sampler.wait_first()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    stream = torch.cuda.current_stream(dev)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    host_t0 = time.time()
+    r0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    host_t1 = time.time()
+    clocks = sampler.summary(host_t0, host_t1)
+    sampler.stop()
+    region_ms = r0.elapsed_time(r1)
+    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    peak, peak_src = measured_hbm_peak()
+    achieved = step_bytes / (kernel_ms * 1e-3) / 1e9
+    # the fp64 oracle on a bounded sample of rows, one thread
+    cpu = None
+    if not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_limits
+
+        from oracle.gdr_oracle import linear_attention_gate as oracle_gate
+        a64 = x["a"].reshape(-1, shape[-1]).double().numpy()
+        b64 = x["b"].reshape(-1, shape[-1]).double().numpy()
+        dtb, dsc = x["dt_bias"].double().numpy(), x["decay_scale"].double().numpy()
+        rows = min(a64.shape[0], 4096)
+        done, t_cpu = 0, 0.0
+        with threadpool_limits(limits=1):
+            while t_cpu < args.cpu_seconds:
+                lo = (done // shape[-1]) % a64.shape[0]
+                t0 = time.perf_counter()
+                oracle_gate(a64[lo:lo + rows], dtb, dsc, b64[lo:lo + rows])
+                t_cpu += time.perf_counter() - t0
+                done += rows * shape[-1]
+        cpu = {"value": done / t_cpu, "unit": "elements/s", "cores": 1, "kind": "oracle",
+               "sample": f"{rows}-row chunks of the same tensor for {t_cpu:.1f} s"}
+    line = {
+        "metric": "LinearAttentionGate elements/s (standalone gate op)",
+        "op": "gate", "value": n * K / (region_ms * 1e-3), "unit": "elements/s", "n_gpus": 1,
+        "steps": K, "warmup": args.warmup, "ms_per_step": region_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": args.gate_dtype, "data": "synthetic",
+        "config": {"workload": f"gate_{args.gate_shape}_{args.gate_dtype}", "shape": list(shape),
+                   "beta": True,
+                   "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB per step vs 126 MiB "
+                         "L2, no flush" if step_bytes > 126 * 2**20 else
+                         f"{step_bytes / 1e6:.1f} MB per step, within L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_src} copy bandwidth",
+                     "kernel": "gdr::gate_vec_kernel", "kernel_ms": kernel_ms,
+                     "bytes_per_launch": step_bytes, "traffic": None},
+        "e2e": None, "gpu_launches": K, "clocks": clocks, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -474,10 +562,23 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--op", choices=("decode", "gate"), default="decode",
+                    help="decode: the decode step (the default line); gate: the standalone "
+                         "LinearAttentionGate op, a line of its own")
+    ap.add_argument("--gate-shape", default="32768x8x64",
+                    help="shape of a and b for --op gate, heads last")
+    ap.add_argument("--gate-dtype", choices=("f32", "f16", "bf16"), default="bf16")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "gdr":
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.op == "gate":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "op": "gate",
+                              "unavailable": "the gate op's reference is the oracle; "
+                                             "see the cpu_baseline key of the gate line"}))
+        else:
+            run_gate(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gdr(args)

@@ -3,15 +3,16 @@
 The compute path is the C-ABI library ``libgdr.so`` built from ``csrc/``; the
 Python functions here only marshal torch tensors into it. Importing the
 package does not load the library: the first use of ``decode``,
-``decode_gated`` or ``lib`` does, and raises if it is missing (there is no CPU
-fallback).
+``decode_gated``, ``linear_attention_gate`` or ``lib`` does, and raises if it is
+missing (there is no CPU fallback).
 """
 from __future__ import annotations
 
-__all__ = ["decode", "decode_gated", "device_error", "GdrError", "lib", "library_path"]
+__all__ = ["decode", "decode_gated", "linear_attention_gate", "device_error", "GdrError", "lib",
+           "library_path"]
 
-_LAZY = {"decode", "decode_gated", "device_error", "GdrError", "lib", "library_path",
-         "STATUS_NAMES"}
+_LAZY = {"decode", "decode_gated", "linear_attention_gate", "device_error", "GdrError", "lib",
+         "library_path", "STATUS_NAMES"}
 
 
 def __getattr__(name):

@@ -15,7 +15,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["decode", "decode_gated", "device_error", "GdrError", "lib", "library_path",
+__all__ = ["decode", "decode_gated", "linear_attention_gate", "device_error", "GdrError", "lib",
+           "library_path",
            "STATUS_NAMES", "Dims"]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +73,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_abi_version.restype = ctypes.c_int
         L.gdr_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
         L.gdr_device_error.restype = ctypes.c_int
+        P = ctypes.c_void_p
+        L.gdr_linear_attention_gate.argtypes = [P, P, P, P, P, P, ctypes.c_int64, ctypes.c_int32,
+                                                ctypes.c_int, P]
+        L.gdr_linear_attention_gate.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -193,3 +198,56 @@ def decode_gated(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, a:
                                   stream)
     _check(rc)
     return out, state_pool
+
+
+# gdr_dtype values of include/gdr.h
+_GATE_DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+
+def linear_attention_gate(a: torch.Tensor, dt_bias: torch.Tensor, decay_scale: torch.Tensor,
+                          b: Optional[torch.Tensor] = None, want_beta: Optional[bool] = None,
+                          decay: Optional[torch.Tensor] = None,
+                          beta: Optional[torch.Tensor] = None):
+    """The LinearAttentionGate op on its own ("com.microsoft.LinearAttentionGate").
+
+    decay = decay_scale * softplus(a + dt_bias) and, when requested, beta =
+    sigmoid(b), computed in float32 and narrowed to a's dtype (float32, float16
+    or bfloat16). The head axis is the last axis of ``a``; dt_bias and
+    decay_scale are float32 [H]. ``want_beta`` defaults to ``b is not None``;
+    requesting beta without b is an error (the page's rule), while a b given
+    with want_beta=False is accepted and not read. Returns (decay, beta or None).
+    """
+    if not isinstance(a, torch.Tensor) or a.dim() < 1:
+        raise RuntimeError("a must be a tensor of rank >= 1 (heads on the last axis)")
+    device = a.device
+    if device.type != "cuda":
+        raise RuntimeError("all tensors must be on a CUDA device")
+    if a.dtype not in _GATE_DTYPES:
+        raise RuntimeError(f"a must be float32, float16 or bfloat16, got {a.dtype}")
+    if want_beta is None:
+        want_beta = b is not None
+    if want_beta and b is None:
+        raise RuntimeError("beta was requested but b is None")
+    H = a.shape[-1]
+    _need(a, "a", a.dtype, a.shape, device)
+    _need(dt_bias, "dt_bias", torch.float32, (H,), device)
+    _need(decay_scale, "decay_scale", torch.float32, (H,), device)
+    if b is not None:
+        _need(b, "b", a.dtype, a.shape, device)
+    if decay is None:
+        decay = torch.empty_like(a)
+    _need(decay, "decay", a.dtype, a.shape, device)
+    if want_beta:
+        if beta is None:
+            beta = torch.empty_like(a)
+        _need(beta, "beta", a.dtype, a.shape, device)
+    else:
+        beta = None
+    rows = a.numel() // H if H > 0 else 0
+    stream = torch.cuda.current_stream(device).cuda_stream
+    with torch.cuda.device(device):
+        rc = lib().gdr_linear_attention_gate(
+            _ptr(a), _ptr(b if want_beta else None), _ptr(dt_bias), _ptr(decay_scale),
+            _ptr(decay), _ptr(beta), rows, H, _GATE_DTYPES[a.dtype], ctypes.c_void_p(stream))
+    _check(rc)
+    return decay, beta

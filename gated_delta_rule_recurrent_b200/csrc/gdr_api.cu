@@ -18,6 +18,7 @@
 #include "gdr_decode.cuh"
 #include "gdr_decode_chunk.cuh"
 #include "gdr_decode_tma.cuh"
+#include "gdr_gate.cuh"
 
 namespace {
 
@@ -378,6 +379,50 @@ gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gd
   return p;
 }
 
+// ---------------------------------------------------------------- standalone gate
+
+template <int TYPE, bool BETA>
+int launch_gate(const void* a, const void* b, const float* dt_bias, const float* decay_scale,
+                void* decay, void* beta, int64_t n, int H, cudaStream_t stream) {
+  using E = gdr::GateElem<TYPE>;
+  using bits = typename E::bits;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
+  DeviceProps props;
+  int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  constexpr int kThreads = 256;
+  const int64_t max_blocks = static_cast<int64_t>(props.sms) * 8;  // 2048 threads per SM
+  auto blocks_for = [&](int64_t work) {
+    const int64_t blk = (work + kThreads - 1) / kThreads;
+    return static_cast<int>(blk < max_blocks ? blk : max_blocks);
+  };
+  // 16-byte vectors when every tensor allows them; the rest element by element
+  const bool vec = aligned16(a) && aligned16(decay) && (!BETA || (aligned16(b) && aligned16(beta)));
+  const int64_t n_vec = vec ? n / E::kPerVec : 0;
+  if (n_vec > 0)
+    gdr::gate_vec_kernel<TYPE, BETA><<<blocks_for(n_vec), kThreads, 0, stream>>>(
+        static_cast<const uint4*>(a), static_cast<const uint4*>(b), dt_bias, decay_scale,
+        static_cast<uint4*>(decay), static_cast<uint4*>(beta), n_vec, H);
+  const int64_t i_begin = n_vec * E::kPerVec;
+  if (i_begin < n)
+    gdr::gate_scalar_kernel<TYPE, BETA><<<blocks_for(n - i_begin), kThreads, 0, stream>>>(
+        static_cast<const bits*>(a), static_cast<const bits*>(b), dt_bias, decay_scale,
+        static_cast<bits*>(decay), static_cast<bits*>(beta), i_begin, n, H);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  return GDR_OK;
+}
+
+template <int TYPE>
+int launch_gate_any(const void* a, const void* b, const float* dt_bias, const float* decay_scale,
+                    void* decay, void* beta, int64_t n, int H, cudaStream_t stream) {
+  return beta != nullptr
+             ? launch_gate<TYPE, true>(a, b, dt_bias, decay_scale, decay, beta, n, H, stream)
+             : launch_gate<TYPE, false>(a, b, dt_bias, decay_scale, decay, beta, n, H, stream);
+}
+
 int check_common_pointers(const gdr_bf16* query, const gdr_bf16* key, const gdr_bf16* value,
                           gdr_bf16* state_pool, const int32_t* asl, const int32_t* idx,
                           const float* gk, gdr_bf16* out) {
@@ -438,6 +483,31 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
   return dispatch(p, dims->D_k, true, reinterpret_cast<cudaStream_t>(stream));
 }
 
+GDR_API int gdr_linear_attention_gate(const void* a, const void* b, const float* dt_bias,
+                                      const float* decay_scale, void* decay, void* beta,
+                                      int64_t rows, int32_t H, int dtype, gdr_stream_t stream) {
+  if (!a || !dt_bias || !decay_scale || !decay)
+    return fail(GDR_ERR_NULL, "a, dt_bias, decay_scale and decay must not be NULL");
+  if (beta != nullptr && b == nullptr)
+    return fail(GDR_ERR_NULL, "beta was requested but b is NULL");
+  if (rows < 0 || H < 1) return fail(GDR_ERR_DIMS, "rows must be >= 0 and H >= 1");
+  if (rows > (static_cast<int64_t>(1) << 62) / H)
+    return fail(GDR_ERR_DIMS, "rows * H must be below 2^62");
+  if (dtype != GDR_DTYPE_F32 && dtype != GDR_DTYPE_F16 && dtype != GDR_DTYPE_BF16)
+    return fail(GDR_ERR_UNSUPPORTED, "dtype must be GDR_DTYPE_F32, GDR_DTYPE_F16 or GDR_DTYPE_BF16");
+  if (rows == 0) return GDR_OK;
+  const int64_t n = rows * H;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case GDR_DTYPE_F32:
+      return launch_gate_any<gdr::kGateF32>(a, b, dt_bias, decay_scale, decay, beta, n, H, st);
+    case GDR_DTYPE_F16:
+      return launch_gate_any<gdr::kGateF16>(a, b, dt_bias, decay_scale, decay, beta, n, H, st);
+    default:
+      return launch_gate_any<gdr::kGateBF16>(a, b, dt_bias, decay_scale, decay, beta, n, H, st);
+  }
+}
+
 GDR_API const char* gdr_status_string(int status) {
   switch (status) {
     case GDR_OK: return "GDR_OK";
@@ -466,6 +536,6 @@ GDR_API int gdr_device_error(uint32_t* flags, int reset) {
   return GDR_OK;
 }
 
-GDR_API int gdr_abi_version(void) { return 1; }
+GDR_API int gdr_abi_version(void) { return 2; }
 
 }  // extern "C"

@@ -185,3 +185,17 @@ def make_inputs(w, *, seed: Optional[int] = None, poison_padding: bool = False,
         "dt_bias": dt_bias.contiguous(),
         "decay_scale": decay_scale.contiguous(),
     }
+
+
+def make_gate_inputs(shape, dtype=torch.bfloat16, *, seed: int = 2024):
+    """Inputs of the standalone gate op with the gate workload's distributions:
+    a, b ~ N(0, 1) of ``shape`` (heads on the last axis) narrowed to ``dtype``;
+    dt_bias ~ U(0, 1) and decay_scale = -exp(U(-1, 1)), float32 [H]."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    H = shape[-1]
+    a = torch.randn(*shape, generator=gen, dtype=torch.float32).to(dtype)
+    b = torch.randn(*shape, generator=gen, dtype=torch.float32).to(dtype)
+    dt_bias = torch.rand(H, generator=gen, dtype=torch.float32)
+    decay_scale = -torch.exp(torch.rand(H, generator=gen, dtype=torch.float32) * 2.0 - 1.0)
+    return {"a": a, "b": b, "dt_bias": dt_bias, "decay_scale": decay_scale}

@@ -141,6 +141,43 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
                            const float* gk, const int32_t* num_accepted_tokens,
                            float scale_value, gdr_bf16* out, gdr_stream_t stream);
 
+/* Element types of the standalone gate's a, b, decay and beta. */
+typedef enum gdr_dtype {
+  GDR_DTYPE_F32 = 0,  /* float32, one of the gate page's types (Type constraints) */
+  GDR_DTYPE_F16 = 1,  /* float16, the other one */
+  GDR_DTYPE_BF16 = 2  /* bfloat16, the decode op's storage type (an extension) */
+} gdr_dtype;
+
+/*
+ * gdr_linear_attention_gate - the LinearAttentionGate op on its own
+ * ("com.microsoft.LinearAttentionGate", sections Description, Inputs, Outputs
+ * and Type constraints). For every element, in float32:
+ *   decay = decay_scale[h] * softplus(a + dt_bias[h])
+ *   beta  = sigmoid(b)                      (only when beta is requested)
+ * narrowed to `dtype` on store (round to nearest even). h is the index on the
+ * last axis; every leading axis is folded into `rows`.
+ *
+ *   a            [rows, H] of `dtype`
+ *   b            [rows, H] of `dtype`, or NULL; read only when beta is requested
+ *   dt_bias      [H] fp32
+ *   decay_scale  [H] fp32 (for gated DeltaNet, -exp(A_log))
+ *   decay        [rows, H] of `dtype`, written
+ *   beta         [rows, H] of `dtype`, written; NULL when beta is not requested
+ *   rows, H      rows >= 0, 1 <= H
+ *   dtype        a gdr_dtype
+ *   stream       CUDA stream the work is queued on
+ *
+ * All pointers are device memory owned by the caller; any alignment works
+ * (16-byte aligned tensors take the vector path). Errors, checked on the host
+ * before anything is queued: GDR_ERR_NULL if a, dt_bias, decay_scale or decay is
+ * NULL, or if beta is requested without b (the page's rule); GDR_ERR_DIMS for
+ * rows < 0, H < 1 or rows * H >= 2^62; GDR_ERR_UNSUPPORTED for an unknown
+ * dtype. rows = 0 queues nothing. Returns a gdr_status.
+ */
+GDR_API int gdr_linear_attention_gate(const void* a, const void* b, const float* dt_bias,
+                                      const float* decay_scale, void* decay, void* beta,
+                                      int64_t rows, int32_t H, int dtype, gdr_stream_t stream);
+
 /* Static English name of a gdr_status value ("GDR_OK", ...); "unknown status"
  * for other values. Never NULL. */
 GDR_API const char* gdr_status_string(int status);
@@ -160,7 +197,7 @@ GDR_API const char* gdr_last_error(void);
  * counterpart on the pages: every bounded wait of the kernels reports here. */
 GDR_API int gdr_device_error(uint32_t* flags, int reset);
 
-/* Library ABI version, currently 1. */
+/* Library ABI version, currently 2 (2 added gdr_linear_attention_gate). */
 GDR_API int gdr_abi_version(void);
 
 #ifdef __cplusplus

@@ -26,8 +26,8 @@ def declared_symbols():
 
 def test_header_declares_the_entry_points():
     names = declared_symbols()
-    for want in ("gdr_decode", "gdr_gate_fused", "gdr_status_string", "gdr_last_error",
-                 "gdr_abi_version"):
+    for want in ("gdr_decode", "gdr_gate_fused", "gdr_linear_attention_gate",
+                 "gdr_status_string", "gdr_last_error", "gdr_abi_version"):
         assert want in names
     assert len(names) == len(set(names))
 
@@ -49,7 +49,7 @@ def test_status_strings_and_version(built_library):
     from gated_delta_rule_recurrent_b200 import binding
 
     L = binding.lib()
-    assert L.gdr_abi_version() == 1
+    assert L.gdr_abi_version() == 2
     for code, name in binding.STATUS_NAMES.items():
         assert L.gdr_status_string(code).decode() == name
     assert L.gdr_status_string(99).decode() == "unknown status"
@@ -139,3 +139,42 @@ def test_binding_refuses_cpu_tensors(built_library):
         decode(x["query"], x["key"], x["value"], x["beta"], x["state_pool"],
                x["actual_seq_lengths"], x["ssm_state_indices"], x["g"], x["gk"],
                x["num_accepted_tokens"], x["scale_value"])
+
+
+@no_device
+@pytest.mark.parametrize("args,status", [
+    (dict(a=None), GDR_ERR_NULL),
+    (dict(dt_bias=None), GDR_ERR_NULL),
+    (dict(decay_scale=None), GDR_ERR_NULL),
+    (dict(decay=None), GDR_ERR_NULL),
+    (dict(b=None), GDR_ERR_NULL),            # beta requested without b (the gate page's rule)
+    (dict(rows=-1), GDR_ERR_DIMS),
+    (dict(H=0), GDR_ERR_DIMS),
+    (dict(rows=1 << 60, H=8), GDR_ERR_DIMS),  # rows * H >= 2^62
+    (dict(dtype=3), GDR_ERR_UNSUPPORTED),
+    (dict(rows=0), GDR_OK),                  # nothing queued
+])
+def test_gate_host_checks(built_library, args, status):
+    """The standalone gate's argument checks, with placeholder pointers."""
+    from gated_delta_rule_recurrent_b200 import binding
+
+    L = binding.lib()
+    P = ctypes.c_void_p
+    kw = dict(a=P(16), b=P(16), dt_bias=P(16), decay_scale=P(16), decay=P(16), beta=P(16),
+              rows=4, H=8, dtype=2)
+    kw.update(args)
+    rc = L.gdr_linear_attention_gate(kw["a"], kw["b"], kw["dt_bias"], kw["decay_scale"],
+                                     kw["decay"], kw["beta"], kw["rows"], kw["H"], kw["dtype"],
+                                     None)
+    assert rc == status, L.gdr_last_error().decode()
+
+
+@no_device
+def test_gate_without_beta_accepts_missing_b(built_library):
+    """b may be absent when beta is not requested (checked without a device:
+    rows = 0 queues nothing)."""
+    from gated_delta_rule_recurrent_b200 import binding
+
+    L = binding.lib()
+    P = ctypes.c_void_p
+    assert L.gdr_linear_attention_gate(P(16), None, P(16), P(16), P(16), None, 0, 8, 0, None) == 0
