@@ -97,6 +97,16 @@ constexpr int kMaxDevices = 64;
 #define GDR_MAX_STAGES 6
 #endif
 constexpr int kMaxStages = GDR_MAX_STAGES;
+// Single-token kernel: at most this many co-resident CTAs per SM, and the
+// widest tile that still gives every SM at least GDR_MIN_TILES_PER_SM tiles
+// (fewer, larger tiles leave a persistent CTA too few tiles to keep its
+// stage ring busy; 16 measured best on the 64-item, 128x128 workload).
+#ifndef GDR_MAX_CTAS_PER_SM
+#define GDR_MAX_CTAS_PER_SM 6
+#endif
+#ifndef GDR_MIN_TILES_PER_SM
+#define GDR_MIN_TILES_PER_SM 16
+#endif
 
 struct DeviceProps {
   int sms = 0;
@@ -155,7 +165,7 @@ int launch_config(int dev, int T, const DeviceProps& props, LaunchConfig* out) {
   // shared-memory budget those CTAs split.
   const int regs_per_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
   int ctas = 65536 / (regs_per_warp * (Shape::kThreads / 32));
-  ctas = ctas < 1 ? 1 : (ctas > 4 ? 4 : ctas);
+  ctas = ctas < 1 ? 1 : (ctas > GDR_MAX_CTAS_PER_SM ? GDR_MAX_CTAS_PER_SM : ctas);
   LaunchConfig c;
   for (; ctas >= 1; --ctas) {
     const int stage_bytes = gdr::stage_layout<DK, VS, R>(T).bytes;
@@ -328,8 +338,9 @@ const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
 }
 
 // Column-slice width: the widest width that divides D_v and still gives every
-// SM a tile, else the narrowest one; a width whose stage ring does not fit in
-// shared memory (long T) falls back to the next narrower one.
+// SM GDR_MIN_TILES_PER_SM tiles, else the narrowest one; a width whose stage
+// ring does not fit in shared memory (long T) falls back to the next narrower
+// one.
 int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
@@ -344,7 +355,9 @@ int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, cudaStream_t strea
   for (int i = 0; i < n; ++i) {
     if (p.D_v % ks[i].vs != 0) continue;
     first = i;
-    if (static_cast<long long>(p.B) * p.H_v * (p.D_v / ks[i].vs) >= props.sms) break;
+    if (static_cast<long long>(p.B) * p.H_v * (p.D_v / ks[i].vs) >=
+        static_cast<long long>(GDR_MIN_TILES_PER_SM) * props.sms)
+      break;
   }
   if (first < 0) return fail(GDR_ERR_UNSUPPORTED, "no tile width divides D_v");
   for (int i = first; i < n; ++i) {
