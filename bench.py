@@ -70,9 +70,9 @@ def kernel_source_hash():
     return h.hexdigest()
 
 
-def recorded_traffic():
+def recorded_traffic(workload_name, layout):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    this workload and layout with the current kernel source; else None."""
     try:
         rec = {}
         with open(TRAFFIC_RECORD) as f:
@@ -81,6 +81,8 @@ def recorded_traffic():
                     k, v = line.split(":", 1)
                     rec[k.strip()] = v.strip()
         if rec.get("kernel_source_sha256") != kernel_source_hash():
+            return None
+        if rec.get("workload") != workload_name or rec.get("state_layout", "kv") != layout:
             return None
         return int(float(rec["dram_bytes_per_launch"]))
     except Exception:
@@ -292,6 +294,8 @@ def run_gdr(args):
     # Each rank decodes its own batch: independent sequences and pool slots.
     x = workloads.make_inputs(w, seed=distributed.rank_seed(w.seed, rank))
     xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    if args.layout == "vk":  # the same state, stored [pool, H_v, D_v, D_k]
+        xd["state_pool"] = xd["state_pool"].transpose(2, 3).contiguous()
     out = torch.empty(w.B, w.H_v, w.T, w.D_v, dtype=torch.bfloat16, device=dev)
     lengths = x["actual_seq_lengths"].tolist()
     n_tokens = int(sum(min(max(L, 0), w.T) for L in lengths))
@@ -305,11 +309,13 @@ def run_gdr(args):
             gdr.decode_gated(z["query"], z["key"], z["value"], z["a"], z["b"],
                              z["dt_bias"], z["decay_scale"], z["state_pool"],
                              z["actual_seq_lengths"], z["ssm_state_indices"], z["gk"],
-                             z["num_accepted_tokens"], z["scale_value"], out=o)
+                             z["num_accepted_tokens"], z["scale_value"], out=o,
+                             state_layout=args.layout)
         else:
             gdr.decode(z["query"], z["key"], z["value"], z["beta"], z["state_pool"],
                        z["actual_seq_lengths"], z["ssm_state_indices"], z["g"], z["gk"],
-                       z["num_accepted_tokens"], z["scale_value"], out=o)
+                       z["num_accepted_tokens"], z["scale_value"], out=o,
+                       state_layout=args.layout)
 
     def barrier():
         if world > 1:
@@ -392,6 +398,8 @@ def run_gdr(args):
             "D_k": w.D_k, "D_v": w.D_v, "pool": w.pool,
             "gate": "fused" if gated else "none",
             "storage": "bf16 state/q/k/v/out, fp32 g/gk",
+            "state_layout": "[pool, H_v, D_k, D_v]" if args.layout == "kv"
+                            else "[pool, H_v, D_v, D_k]",
             "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB per step vs "
                   f"{L2_BYTES / 2**20:.0f} MiB L2, no flush",
             "parallelism": f"{world} independent rank(s), no collective",
@@ -401,8 +409,9 @@ def run_gdr(args):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth",
-            "kernel": "gdr::decode_tma_kernel", "kernel_ms": kernel_ms,
-            "bytes_per_launch": step_bytes, "traffic": recorded_traffic(),
+            "kernel": ("gdr::decode_tma_kernel" if w.T == 1 and args.layout == "kv"
+                       else "gdr::decode_chunk_kernel"), "kernel_ms": kernel_ms,
+            "bytes_per_launch": step_bytes, "traffic": recorded_traffic(w.name, args.layout),
         },
         "e2e": e2e,
         "gpu_launches": launches,
@@ -568,6 +577,9 @@ def main():
     ap.add_argument("--gate-shape", default="32768x8x64",
                     help="shape of a and b for --op gate, heads last")
     ap.add_argument("--gate-dtype", choices=("f32", "f16", "bf16"), default="bf16")
+    ap.add_argument("--layout", choices=("kv", "vk"), default="kv",
+                    help="state pool layout: kv = [pool, H_v, D_k, D_v] (the op page's), "
+                         "vk = [pool, H_v, D_v, D_k]")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "gdr":
         raise SystemExit("--warmup must be >= 3")

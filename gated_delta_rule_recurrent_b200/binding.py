@@ -34,8 +34,9 @@ class GdrError(RuntimeError):
 
 
 class Dims(ctypes.Structure):
+    """gdr_dims; ``layout`` is 0 (GDR_LAYOUT_KV) unless given."""
     _fields_ = [(n, ctypes.c_int32)
-                for n in ("B", "T", "H_qk", "H_v", "D_k", "D_v", "pool_size")]
+                for n in ("B", "T", "H_qk", "H_v", "D_k", "D_v", "pool_size", "layout")]
 
 
 _P = ctypes.c_void_p
@@ -113,8 +114,12 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+# gdr_state_layout values of include/gdr.h
+_LAYOUTS = {"kv": 0, "vk": 1}
+
+
 def _common(query, key, value, state_pool, actual_seq_lengths, ssm_state_indices, gk,
-            num_accepted_tokens, out):
+            num_accepted_tokens, out, state_layout="kv"):
     if not isinstance(query, torch.Tensor) or query.dim() != 4:
         raise RuntimeError("query must be a 4-D tensor [B, H_qk, T, D_k]")
     device = query.device
@@ -124,14 +129,19 @@ def _common(query, key, value, state_pool, actual_seq_lengths, ssm_state_indices
     if not isinstance(value, torch.Tensor) or value.dim() != 4:
         raise RuntimeError("value must be a 4-D tensor [B, H_v, T, D_v]")
     H_v, D_v = value.shape[1], value.shape[3]
+    if state_layout not in _LAYOUTS:
+        raise RuntimeError('state_layout must be "kv" ([pool, H_v, D_k, D_v]) or "vk" '
+                           '([pool, H_v, D_v, D_k])')
     if not isinstance(state_pool, torch.Tensor) or state_pool.dim() != 4:
-        raise RuntimeError("state_pool must be a 4-D tensor [pool, H_v, D_k, D_v]")
+        raise RuntimeError("state_pool must be a 4-D tensor [pool, H_v, D_k, D_v] "
+                           "(or [pool, H_v, D_v, D_k] for state_layout='vk')")
     P = state_pool.shape[0]
     bf16, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     _need(query, "query", bf16, (B, H_qk, T, D_k), device)
     _need(key, "key", bf16, (B, H_qk, T, D_k), device)
     _need(value, "value", bf16, (B, H_v, T, D_v), device)
-    _need(state_pool, "state_pool", bf16, (P, H_v, D_k, D_v), device)
+    _need(state_pool, "state_pool", bf16,
+          (P, H_v, D_k, D_v) if state_layout == "kv" else (P, H_v, D_v, D_k), device)
     _need(actual_seq_lengths, "actual_seq_lengths", i32, (B,), device)
     _need(ssm_state_indices, "ssm_state_indices", i32, (B,), device)
     _need(gk, "gk", f32, (B, H_v, T, D_k), device)
@@ -141,7 +151,7 @@ def _common(query, key, value, state_pool, actual_seq_lengths, ssm_state_indices
         out = torch.empty((B, H_v, T, D_v), dtype=bf16, device=device)
     else:
         _need(out, "out", bf16, (B, H_v, T, D_v), device)
-    dims = Dims(B, T, H_qk, H_v, D_k, D_v, P)
+    dims = Dims(B, T, H_qk, H_v, D_k, D_v, P, _LAYOUTS[state_layout])
     stream = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
     return device, dims, out, stream
 
@@ -150,15 +160,19 @@ def decode(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, beta: to
            state_pool: torch.Tensor, actual_seq_lengths: torch.Tensor,
            ssm_state_indices: torch.Tensor, g: torch.Tensor, gk: torch.Tensor,
            num_accepted_tokens: Optional[torch.Tensor] = None, scale_value: float = 1.0, *,
-           out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+           out: Optional[torch.Tensor] = None,
+           state_layout: str = "kv") -> Tuple[torch.Tensor, torch.Tensor]:
     """recurrent_gated_delta_rule decode step through ``gdr_decode``.
 
     Argument order and defaults follow the op's page. ``state_pool`` is
     updated in place and returned as the second result (the page's
-    ``state_out``). Queued on the current CUDA stream; no synchronisation.
+    ``state_out``). ``state_layout`` "vk" takes the pool as [pool, H_v, D_v,
+    D_k] (k contiguous) instead of the page's [pool, H_v, D_k, D_v]. Queued on
+    the current CUDA stream; no synchronisation.
     """
     device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
-                                        ssm_state_indices, gk, num_accepted_tokens, out)
+                                        ssm_state_indices, gk, num_accepted_tokens, out,
+                                        state_layout)
     B, H_v, T = dims.B, dims.H_v, dims.T
     _need(beta, "beta", torch.bfloat16, (B, H_v, T), device)
     _need(g, "g", torch.float32, (B, H_v, T), device)
@@ -176,14 +190,17 @@ def decode_gated(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, a:
                  state_pool: torch.Tensor, actual_seq_lengths: torch.Tensor,
                  ssm_state_indices: torch.Tensor, gk: torch.Tensor,
                  num_accepted_tokens: Optional[torch.Tensor] = None, scale_value: float = 1.0,
-                 *, out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                 *, out: Optional[torch.Tensor] = None,
+                 state_layout: str = "kv") -> Tuple[torch.Tensor, torch.Tensor]:
     """Decode step with the LinearAttentionGate prologue fused, through ``gdr_gate_fused``.
 
     ``a`` and ``b`` are [B, T, H_v] bf16; ``dt_bias`` and ``decay_scale`` are
-    [H_v] fp32. g and beta are computed inside the kernel.
+    [H_v] fp32. g and beta are computed inside the kernel. ``state_layout`` as
+    for ``decode``.
     """
     device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
-                                        ssm_state_indices, gk, num_accepted_tokens, out)
+                                        ssm_state_indices, gk, num_accepted_tokens, out,
+                                        state_layout)
     B, H_v, T = dims.B, dims.H_v, dims.T
     _need(a, "a", torch.bfloat16, (B, T, H_v), device)
     _need(b, "b", torch.bfloat16, (B, T, H_v), device)

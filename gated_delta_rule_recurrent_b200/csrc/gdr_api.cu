@@ -48,9 +48,12 @@ int check_dims(const gdr_dims* d) {
   // Grid size: B * H_v * (D_v / 64) CTAs must fit a 31-bit grid dimension.
   const long long ctas = static_cast<long long>(d->B) * d->H_v * (d->D_v / gdr::kSliceCols);
   if (ctas > 0x7fffffffLL) return fail(GDR_ERR_DIMS, "B * H_v * D_v / 64 exceeds 2^31 - 1");
+  if (d->layout != GDR_LAYOUT_KV && d->layout != GDR_LAYOUT_VK)
+    return fail(GDR_ERR_DIMS, "layout must be GDR_LAYOUT_KV or GDR_LAYOUT_VK");
   // TMA row coordinates of the pool are 32-bit signed.
-  if (static_cast<long long>(d->pool_size) * d->H_v * d->D_k > 0x7fffffffLL)
-    return fail(GDR_ERR_UNSUPPORTED, "pool_size * H_v * D_k exceeds 2^31 - 1");
+  const long long rows_per_slot = d->layout == GDR_LAYOUT_VK ? d->D_v : d->D_k;
+  if (static_cast<long long>(d->pool_size) * d->H_v * rows_per_slot > 0x7fffffffLL)
+    return fail(GDR_ERR_UNSUPPORTED, "pool_size * H_v * (rows per head) exceeds 2^31 - 1");
   return GDR_OK;
 }
 
@@ -70,18 +73,24 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// The pool seen as a 3-D bf16 array [D_v / 64 column blocks][pool * H_v * D_k
-// rows][64 columns] (row stride D_v * 2 bytes, block stride 128 bytes). One
-// box {64, D_k, VS / 64} is a whole tile and lands in shared memory as
-// [block][row][64 columns] with the 128-byte swizzle: within each 128-byte
-// row segment, 16-byte chunk c is stored at position c ^ (row % 8).
-int encode_pool_map(const gdr::DecodeParams& p, int DK, int VS, CUtensorMap* map) {
+// The pool seen as a 3-D bf16 array [column blocks of 64][rows][64 columns]
+// (row stride = row length * 2 bytes, block stride 128 bytes); one box is a
+// whole tile and lands in shared memory as [block][row][64 columns] with the
+// 128-byte swizzle: within each 128-byte row segment, 16-byte chunk c is
+// stored at position c ^ (row % 8).
+//   KV pool [pool, H_v, D_k, D_v]: rows of D_v, box {64, D_k, VS / 64};
+//   VK pool [pool, H_v, D_v, D_k]: rows of D_k, box {64, VS, D_k / 64}.
+int encode_pool_map(const gdr::DecodeParams& p, int DK, int VS, bool vk, CUtensorMap* map) {
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return fail(GDR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t gdim[3] = {64, static_cast<cuuint64_t>(p.pool_size) * p.H_v * DK,
-                              static_cast<cuuint64_t>(p.D_v / 64)};
-  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(p.D_v) * 2, 128};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(DK), static_cast<cuuint32_t>(VS / 64)};
+  const int row_len = vk ? DK : p.D_v;          // entries per pool row
+  const int rows_per_head = vk ? p.D_v : DK;
+  const int box_rows = vk ? VS : DK;
+  const cuuint64_t gdim[3] = {64, static_cast<cuuint64_t>(p.pool_size) * p.H_v * rows_per_head,
+                              static_cast<cuuint64_t>(row_len / 64)};
+  const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(row_len) * 2, 128};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows),
+                             static_cast<cuuint32_t>((vk ? DK : VS) / 64)};
   const cuuint32_t estride[3] = {1, 1, 1};
   const CUresult cr = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                              const_cast<uint16_t*>(p.state_pool), gdim, gstride, box, estride,
@@ -210,7 +219,7 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   const int ctas_per_sm = cfg.ctas_per_sm;
 
   CUtensorMap map;
-  rc = encode_pool_map(p, DK, VS, &map);
+  rc = encode_pool_map(p, DK, VS, false, &map);
   if (rc != GDR_OK) return rc;
 
   const int n_tiles = p.B * p.H_v * (p.D_v / VS);
@@ -239,7 +248,7 @@ struct ChunkConfig {
 
 // One persistent CTA per SM: as many stages as shared memory holds, and one
 // consumer group fewer than stages (so no group waits two phases ahead).
-template <int DK, int VS, bool GATED>
+template <int DK, int VS, bool GATED, bool VK>
 int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   static ChunkConfig cache[kMaxDevices][gdr::kMaxT + 1];
   static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
@@ -247,7 +256,7 @@ int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
     *out = cache[dev][T];
     return GDR_OK;
   }
-  auto kernel = gdr::decode_chunk_kernel<DK, VS, GATED>;
+  auto kernel = gdr::decode_chunk_kernel<DK, VS, GATED, VK>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          props.smem_optin);
   if (err == cudaSuccess)
@@ -260,7 +269,7 @@ int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   int n = (props.smem_optin - 1024 - gdr::kChunkBarriers * 8 * kMaxStagesChunk) / stage_bytes;
   n = n > kMaxStagesChunk ? kMaxStagesChunk : n;
   if (n < 2) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
-  constexpr int cwt = gdr::ChunkShape<DK, VS>::kWarpsPerTile;
+  constexpr int cwt = gdr::ChunkShape<DK, VS, VK>::kWarpsPerTile;
   int groups = n - 1;
   const int max_groups = (gdr::kChunkMaxThreads / 32 - 1 - gdr::kChunkFinalizers) / cwt;
   groups = groups > max_groups ? max_groups : groups;
@@ -279,7 +288,7 @@ int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   return GDR_OK;
 }
 
-template <int DK, int VS, bool GATED>
+template <int DK, int VS, bool GATED, bool VK>
 int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -288,15 +297,15 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   ChunkConfig cfg;
-  rc = chunk_config<DK, VS, GATED>(dev, p.T, props, &cfg);
+  rc = chunk_config<DK, VS, GATED, VK>(dev, p.T, props, &cfg);
   if (rc != GDR_OK) return rc;
   CUtensorMap map;
-  rc = encode_pool_map(p, DK, VS, &map);
+  rc = encode_pool_map(p, DK, VS, VK, &map);
   if (rc != GDR_OK) return rc;
   const int n_tiles = p.B * p.H_v * (p.D_v / VS);
   const int grid = n_tiles < props.sms ? n_tiles : props.sms;
-  gdr::decode_chunk_kernel<DK, VS, GATED><<<grid, cfg.threads, cfg.smem, stream>>>(map, p, n_tiles,
-                                                                                  cfg.n_stages);
+  gdr::decode_chunk_kernel<DK, VS, GATED, VK><<<grid, cfg.threads, cfg.smem, stream>>>(
+      map, p, n_tiles, cfg.n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
@@ -317,7 +326,7 @@ struct SliceKernel {
 // full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls use
 // the chunked kernel (64 columns per consumer warp).
 template <bool GATED>
-const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
+const SliceKernel* slice_kernels(int D_k, bool one, bool vk, int* n) {
   static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED>},
                                         {256, launch_tma<64, 256, 8, GATED>},
                                         {128, launch_tma<64, 128, 8, GATED>},
@@ -325,10 +334,19 @@ const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
   static const SliceKernel k128_one[] = {{256, launch_tma<128, 256, 16, GATED>},
                                          {128, launch_tma<128, 128, 16, GATED>},
                                          {64, launch_tma<128, 64, 16, GATED>}};
-  static const SliceKernel k64_many[] = {{128, launch_chunk<64, 128, GATED>},
-                                         {64, launch_chunk<64, 64, GATED>}};
-  static const SliceKernel k128_many[] = {{128, launch_chunk<128, 128, GATED>},
-                                          {64, launch_chunk<128, 64, GATED>}};
+  static const SliceKernel k64_many[] = {{128, launch_chunk<64, 128, GATED, false>},
+                                         {64, launch_chunk<64, 64, GATED, false>}};
+  static const SliceKernel k128_many[] = {{128, launch_chunk<128, 128, GATED, false>},
+                                          {64, launch_chunk<128, 64, GATED, false>}};
+  // k-contiguous pools: the chunked kernel for every T (one token is L = 1)
+  static const SliceKernel k64_vk[] = {{128, launch_chunk<64, 128, GATED, true>},
+                                       {64, launch_chunk<64, 64, GATED, true>}};
+  static const SliceKernel k128_vk[] = {{128, launch_chunk<128, 128, GATED, true>},
+                                        {64, launch_chunk<128, 64, GATED, true>}};
+  if (vk) {
+    *n = 2;
+    return D_k == 64 ? k64_vk : k128_vk;
+  }
   if (D_k == 64) {
     *n = one ? 4 : 2;
     return one ? k64_one : k64_many;
@@ -341,7 +359,7 @@ const SliceKernel* slice_kernels(int D_k, bool one, int* n) {
 // SM GDR_MIN_TILES_PER_SM tiles, else the narrowest one; a width whose stage
 // ring does not fit in shared memory (long T) falls back to the next narrower
 // one.
-int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, cudaStream_t stream) {
+int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, bool vk, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
   DeviceProps props;
@@ -349,8 +367,8 @@ int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, cudaStream_t strea
   if (rc != GDR_OK) return rc;
   int n = 0;
   const bool one = p.T == 1;
-  const SliceKernel* ks =
-      gated ? slice_kernels<true>(D_k, one, &n) : slice_kernels<false>(D_k, one, &n);
+  const SliceKernel* ks = gated ? slice_kernels<true>(D_k, one, vk, &n)
+                                : slice_kernels<false>(D_k, one, vk, &n);
   int first = -1;
   for (int i = 0; i < n; ++i) {
     if (p.D_v % ks[i].vs != 0) continue;
@@ -469,7 +487,8 @@ GDR_API int gdr_decode(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf
                                     ssm_state_indices, gk, scale_value, out);
   p.beta = beta;
   p.g = g;
-  return dispatch(p, dims->D_k, false, reinterpret_cast<cudaStream_t>(stream));
+  return dispatch(p, dims->D_k, false, dims->layout == GDR_LAYOUT_VK,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
@@ -493,7 +512,8 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
   p.gate_b = b;
   p.dt_bias = dt_bias;
   p.decay_scale = decay_scale;
-  return dispatch(p, dims->D_k, true, reinterpret_cast<cudaStream_t>(stream));
+  return dispatch(p, dims->D_k, true, dims->layout == GDR_LAYOUT_VK,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 GDR_API int gdr_linear_attention_gate(const void* a, const void* b, const float* dt_bias,
@@ -549,6 +569,6 @@ GDR_API int gdr_device_error(uint32_t* flags, int reset) {
   return GDR_OK;
 }
 
-GDR_API int gdr_abi_version(void) { return 2; }
+GDR_API int gdr_abi_version(void) { return 3; }
 
 }  // extern "C"

@@ -86,12 +86,28 @@ constexpr int kChunkMaxThreads = GDR_CHUNK_MAX_THREADS;
 #endif
 constexpr int kChunkMaxSubTokens = GDR_CHUNK_SWEEP_TOKENS;  // tokens per pass-1 sweep
 
-template <int DK, int VS>
+// Rows of the state per consumer thread in the k-contiguous layout (VK): the
+// per-row vectors a thread reads are shared by its rows.
+#ifndef GDR_VK_ROWS
+#define GDR_VK_ROWS 2
+#endif
+#ifndef GDR_VK_SWEEP_TOKENS
+#define GDR_VK_SWEEP_TOKENS 4
+#endif
+constexpr int kVkRowsPerThread = GDR_VK_ROWS;
+constexpr int kVkSweepTokens = GDR_VK_SWEEP_TOKENS;
+
+// VK: the pool is [pool, H_v, D_v, D_k] (k contiguous) and the tile is VS
+// rows j (value columns) x D_k; otherwise [pool, H_v, D_k, D_v] and the tile
+// is D_k rows x VS columns.
+template <int DK, int VS, bool VK = false>
 struct ChunkShape {
-  static constexpr int kWarpsPerTile = VS / kChunkWarpCols;
+  static constexpr int kWarpsPerTile = VK ? VS / (32 * kVkRowsPerThread) : VS / kChunkWarpCols;
   static constexpr int kStateBytes = DK * VS * 2;
   static_assert(DK == 64 || DK == 128, "D_k must be 64 or 128");
   static_assert(VS == 64 || VS == 128, "64- or 128-column tiles");
+  static_assert(kWarpsPerTile >= 1 && kWarpsPerTile * (VK ? 32 * kVkRowsPerThread : 32) == VS,
+                "a tile must be covered by whole consumer warps");
 };
 
 // Shared memory: n_stages state tiles (DK x VS bf16, 128-byte swizzled, each
@@ -485,6 +501,169 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const uint8_t* 
   }
 }
 
+// ---------------------------------------------------------------- consumers, k-contiguous pool
+
+// One tile with L = LC tokens in the VK layout: the staged tile holds VS rows
+// j (value columns of the state) of D_k entries each, as [D_k / 64][VS][64]
+// with the 128-byte swizzle. Thread `tj` of the group owns rows tj + r * VS /
+// kVkRowsPerThread; its column sums over i, its solve and its update need no
+// other thread. `dst` points at row 0 of the slot's slice; `out_t0` at token
+// 0, column 0 of the tile's output.
+template <int DK, int VS, int LC>
+__device__ __forceinline__ void chunk_consume_vk(const uint8_t* st, const uint8_t* vb,
+                                                 const ChunkLayout& lay, int tj, uint16_t* dst,
+                                                 uint16_t* out_t0, int D_v) {
+  constexpr int R = kVkRowsPerThread;
+  constexpr int RS = VS / R;  // row stride between a thread's rows
+  const float* su = reinterpret_cast<const float*>(vb + lay.u);
+  const float* sw = reinterpret_cast<const float*>(vb + lay.w);
+  const float* se = reinterpret_cast<const float*>(vb + lay.e);
+  const float* sc = reinterpret_cast<const float*>(vb + lay.c);
+  // byte offset of (row tj + r RS, columns [8 c8, 8 c8 + 8)) is off[r] + c8-term:
+  // the chunk index within a 128-byte segment is c8 % 8, swizzled by row % 8
+  auto chunk = [&](int r, int c8) -> uint4 {
+    const int j = tj + r * RS;
+    return *reinterpret_cast<const uint4*>(st + swz_offset<VS>(j, 8 * c8));
+  };
+  // ---- pass 1: m_t = S_0^T u_t and p_t = S_0^T w_t for this thread's rows,
+  // packed fp32 pairs over (i, i + 1), two accumulators per vector
+  float ms[R][LC], ps[R][LC];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int t = 0; t < LC; ++t) ms[r][t] = ps[r][t] = 0.0f;
+  constexpr int SW = LC < kVkSweepTokens ? LC : kVkSweepTokens;
+#pragma unroll
+  for (int t0 = 0; t0 < LC; t0 += SW) {  // sweeps of at most SW tokens
+    unsigned long long acc[R][2 * SW][2];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int v = 0; v < 2 * SW; ++v) acc[r][v][0] = acc[r][v][1] = 0ull;
+#pragma unroll 1
+    for (int c8 = 0; c8 < DK / 8; ++c8) {
+      unsigned long long x[R][4];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint4 w = chunk(r, c8);
+        x[r][0] = pk(bf16_lo(w.x), bf16_hi(w.x));
+        x[r][1] = pk(bf16_lo(w.y), bf16_hi(w.y));
+        x[r][2] = pk(bf16_lo(w.z), bf16_hi(w.z));
+        x[r][3] = pk(bf16_lo(w.w), bf16_hi(w.w));
+      }
+#pragma unroll
+      for (int tt = 0; tt < SW; ++tt) {
+        if (t0 + tt < LC) {
+          const ulonglong2 u01 = *reinterpret_cast<const ulonglong2*>(su + (t0 + tt) * DK + 8 * c8);
+          const ulonglong2 u23 =
+              *reinterpret_cast<const ulonglong2*>(su + (t0 + tt) * DK + 8 * c8 + 4);
+          const ulonglong2 w01 = *reinterpret_cast<const ulonglong2*>(sw + (t0 + tt) * DK + 8 * c8);
+          const ulonglong2 w23 =
+              *reinterpret_cast<const ulonglong2*>(sw + (t0 + tt) * DK + 8 * c8 + 4);
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            acc[r][tt][0] = fma2(x[r][0], u01.x, acc[r][tt][0]);
+            acc[r][tt][1] = fma2(x[r][1], u01.y, acc[r][tt][1]);
+            acc[r][tt][0] = fma2(x[r][2], u23.x, acc[r][tt][0]);
+            acc[r][tt][1] = fma2(x[r][3], u23.y, acc[r][tt][1]);
+            acc[r][SW + tt][0] = fma2(x[r][0], w01.x, acc[r][SW + tt][0]);
+            acc[r][SW + tt][1] = fma2(x[r][1], w01.y, acc[r][SW + tt][1]);
+            acc[r][SW + tt][0] = fma2(x[r][2], w23.x, acc[r][SW + tt][0]);
+            acc[r][SW + tt][1] = fma2(x[r][3], w23.y, acc[r][SW + tt][1]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int tt = 0; tt < SW; ++tt) {
+        if (t0 + tt < LC) {
+          const float2 a0 = upk(acc[r][tt][0]), a1 = upk(acc[r][tt][1]);
+          const float2 b0 = upk(acc[r][SW + tt][0]), b1 = upk(acc[r][SW + tt][1]);
+          ms[r][t0 + tt] = (a0.x + a0.y) + (a1.x + a1.y);
+          ps[r][t0 + tt] = (b0.x + b0.y) + (b1.x + b1.y);
+        }
+      }
+  }
+
+  // ---- delta (unit lower-triangular solve) and o, per row
+  const float* sa = reinterpret_cast<const float*>(vb + lay.a);
+  const float* sb = reinterpret_cast<const float*>(vb + lay.bm);
+  const uint16_t* sv = reinterpret_cast<const uint16_t*>(vb + lay.v);
+  const float* sbeta = reinterpret_cast<const float*>(vb + lay.beta);
+  unsigned long long dd[R][LC];  // {delta_s[j], delta_s[j]}
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int j = tj + r * RS;
+    float dl[LC];
+#pragma unroll
+    for (int t = 0; t < LC; ++t) {
+      float kv = ms[r][t];  // kv_mem_t = S_0^T u_t + sum_{s<t} A_ts delta_s
+#pragma unroll
+      for (int s = 0; s < t; ++s) kv = fmaf(sa[t * 8 + s], dl[s], kv);
+      dl[t] = (bf16_bits_to_f32(sv[t * VS + j]) - kv) * sbeta[t];  // step 3
+      float o = ps[r][t];  // o_t = S_0^T w_t + sum_{s<=t} B_ts delta_s (step 4)
+#pragma unroll
+      for (int s = 0; s <= t; ++s) o = fmaf(sb[t * 8 + s], dl[s], o);
+      out_t0[static_cast<size_t>(t) * D_v + j] = f32_to_bf16_bits(o);
+      dd[r][t] = pk(dl[t], dl[t]);
+    }
+  }
+
+  // ---- pass 2: S_L = c o S_0 + sum_s e_s delta_s^T, bf16 once, to the slot
+#pragma unroll 1
+  for (int c8 = 0; c8 < DK / 8; ++c8) {
+    const ulonglong2 c01 = *reinterpret_cast<const ulonglong2*>(sc + 8 * c8);
+    const ulonglong2 c23 = *reinterpret_cast<const ulonglong2*>(sc + 8 * c8 + 4);
+    unsigned long long n[R][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint4 w = chunk(r, c8);
+      n[r][0] = mul2(pk(bf16_lo(w.x), bf16_hi(w.x)), c01.x);
+      n[r][1] = mul2(pk(bf16_lo(w.y), bf16_hi(w.y)), c01.y);
+      n[r][2] = mul2(pk(bf16_lo(w.z), bf16_hi(w.z)), c23.x);
+      n[r][3] = mul2(pk(bf16_lo(w.w), bf16_hi(w.w)), c23.y);
+    }
+#pragma unroll
+    for (int s = 0; s < LC; ++s) {
+      const ulonglong2 e01 = *reinterpret_cast<const ulonglong2*>(se + s * DK + 8 * c8);
+      const ulonglong2 e23 = *reinterpret_cast<const ulonglong2*>(se + s * DK + 8 * c8 + 4);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        n[r][0] = fma2(e01.x, dd[r][s], n[r][0]);
+        n[r][1] = fma2(e01.y, dd[r][s], n[r][1]);
+        n[r][2] = fma2(e23.x, dd[r][s], n[r][2]);
+        n[r][3] = fma2(e23.y, dd[r][s], n[r][3]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float2 a = upk(n[r][0]), b = upk(n[r][1]), c = upk(n[r][2]), d = upk(n[r][3]);
+      __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(tj + r * RS) * DK + 8 * c8),
+             make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y), pack_bf16x2(c.x, c.y),
+                        pack_bf16x2(d.x, d.y)));
+    }
+  }
+}
+
+template <int DK, int VS>
+__device__ __forceinline__ void chunk_consume_vk_any(int L, const uint8_t* st, const uint8_t* vb,
+                                                     const ChunkLayout& lay, int tj,
+                                                     uint16_t* dst, uint16_t* out_t0, int D_v) {
+  switch (L) {
+    case 1: chunk_consume_vk<DK, VS, 1>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 2: chunk_consume_vk<DK, VS, 2>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 3: chunk_consume_vk<DK, VS, 3>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 4: chunk_consume_vk<DK, VS, 4>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 5: chunk_consume_vk<DK, VS, 5>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 6: chunk_consume_vk<DK, VS, 6>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 7: chunk_consume_vk<DK, VS, 7>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 8: chunk_consume_vk<DK, VS, 8>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    default: break;
+  }
+}
+
 template <int DK, int VS>
 __device__ __forceinline__ void chunk_consume_any(int L, const uint8_t* st, const uint8_t* vb,
                                                   const ChunkLayout& lay, int c0, int rg, int lane,
@@ -508,11 +687,11 @@ __device__ __forceinline__ void chunk_consume_any(int L, const uint8_t* st, cons
 // warps, then the producer warp; NG = (blockDim.x / 32 - 1 - kChunkFinalizers)
 // / (VS / 32). Requires n_stages >= NG + 1: tiles are finalised in tile order,
 // so a group never waits on a stage two phases ahead of it.
-template <int DK, int VS, bool GATED>
+template <int DK, int VS, bool GATED, bool VK>
 __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     decode_chunk_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                         const int n_tiles, const int n_stages) {
-  using Shape = ChunkShape<DK, VS>;
+  using Shape = ChunkShape<DK, VS, VK>;
   constexpr int CWT = Shape::kWarpsPerTile;
   constexpr int NF = kChunkFinalizers;
   const int T = p.T;
@@ -658,8 +837,12 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
               bulk_load(smem_addr(vb + lay.v + t * VS * 2), vsrc + static_cast<size_t>(t) * p.D_v,
                         VS * 2, vbar);
           }
-          tma_load_3d(smem_addr(smem + stage * Shape::kStateBytes), &pool_map, 0,
-                      (s * p.H_v + h) * DK, slice * VS / 64, sbar);
+          if constexpr (VK)  // VS rows of D_k entries
+            tma_load_3d(smem_addr(smem + stage * Shape::kStateBytes), &pool_map, 0,
+                        (s * p.H_v + h) * p.D_v + slice * VS, 0, sbar);
+          else  // D_k rows of VS entries
+            tma_load_3d(smem_addr(smem + stage * Shape::kStateBytes), &pool_map, 0,
+                        (s * p.H_v + h) * DK, slice * VS / 64, sbar);
         }
         mbar_arrive(sbar);
       }
@@ -694,6 +877,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
   const int rg = lane >> 3;
   const int c0 = gw * kChunkWarpCols + (lane & 7) * 4;  // first tile column of this lane
   const int col = c0 + solved_column(rg);               // the column this lane solves
+  const int tj = gw * 32 + lane;                        // VK: first row of this thread
   for (int it = group; it < n_mine; it += n_groups) {
     const int tile = blockIdx.x + it * gridDim.x;
     const int slice = tile % n_slices;
@@ -719,12 +903,25 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     // out[b, h, t, slice * VS + column]; padded tokens get +0.0
     const size_t bh = static_cast<size_t>(b) * p.H_v + h;
     uint16_t* out_t0 = p.out + bh * T * p.D_v + slice * VS;
-    for (int t = L; t < T; ++t) out_t0[static_cast<size_t>(t) * p.D_v + col] = 0;
+    if constexpr (VK) {
+#pragma unroll
+      for (int r = 0; r < kVkRowsPerThread; ++r)
+        for (int t = L; t < T; ++t)
+          out_t0[static_cast<size_t>(t) * p.D_v + tj + r * (VS / kVkRowsPerThread)] = 0;
+    } else {
+      for (int t = L; t < T; ++t) out_t0[static_cast<size_t>(t) * p.D_v + col] = 0;
+    }
 
     if (L > 0) {
-      uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
-                      slice * VS + c0;
-      chunk_consume_any<DK, VS>(L, st, vb, lay, c0, rg, lane, dst, out_t0, p.D_v);
+      if constexpr (VK) {
+        uint16_t* dst =
+            p.state_pool + ((static_cast<size_t>(s) * p.H_v + h) * p.D_v + slice * VS) * DK;
+        chunk_consume_vk_any<DK, VS>(L, st, vb, lay, tj, dst, out_t0, p.D_v);
+      } else {
+        uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
+                        slice * VS + c0;
+        chunk_consume_any<DK, VS>(L, st, vb, lay, c0, rg, lane, dst, out_t0, p.D_v);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * stage);

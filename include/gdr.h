@@ -71,9 +71,20 @@ typedef uint16_t gdr_bf16;
 /* Same type as cudaStream_t, declared without the CUDA headers. */
 typedef struct CUstream_st* gdr_stream_t;
 
+/* Layout of state_pool. */
+typedef enum gdr_state_layout {
+  /* [pool_size, H_v, D_k, D_v]: the op page's state layout (参数: state), D_v
+   * contiguous. The default. */
+  GDR_LAYOUT_KV = 0,
+  /* [pool_size, H_v, D_v, D_k]: the NPU operator's internal layout (注), D_k
+   * contiguous; the same state, transposed per head. */
+  GDR_LAYOUT_VK = 1
+} gdr_state_layout;
+
 /* Sizes of one call. B batch items, T padded tokens per item, H_qk query/key
  * heads, H_v value heads, D_k key width (state rows), D_v value width (state
- * columns), pool_size slots in state_pool. */
+ * columns), pool_size slots in state_pool, layout a gdr_state_layout (0 when
+ * the struct is zero-initialised). */
 typedef struct gdr_dims {
   int32_t B;
   int32_t T;
@@ -82,6 +93,7 @@ typedef struct gdr_dims {
   int32_t D_k;
   int32_t D_v;
   int32_t pool_size;
+  int32_t layout;
 } gdr_dims;
 
 typedef enum gdr_status {
@@ -101,7 +113,9 @@ typedef enum gdr_status {
  *   key                 [B, H_qk, T, D_k] bf16
  *   value               [B, H_v,  T, D_v] bf16
  *   beta                [B, H_v,  T]      bf16
- *   state_pool          [pool_size, H_v, D_k, D_v] bf16, read and written in place
+ *   state_pool          [pool_size, H_v, D_k, D_v] bf16 (dims->layout = GDR_LAYOUT_KV)
+ *                       or [pool_size, H_v, D_v, D_k] (GDR_LAYOUT_VK), read and
+ *                       written in place
  *   actual_seq_lengths  [B] int32, valid tokens per item
  *   ssm_state_indices   [B] int32, pool slot per item
  *   g                   [B, H_v, T]       fp32
@@ -197,7 +211,8 @@ GDR_API const char* gdr_last_error(void);
  * counterpart on the pages: every bounded wait of the kernels reports here. */
 GDR_API int gdr_device_error(uint32_t* flags, int reset);
 
-/* Library ABI version, currently 2 (2 added gdr_linear_attention_gate). */
+/* Library ABI version, currently 3 (2 added gdr_linear_attention_gate, 3 the
+ * layout field of gdr_dims). */
 GDR_API int gdr_abi_version(void);
 
 #ifdef __cplusplus

@@ -69,18 +69,25 @@ def to_device(x: dict, device="cuda") -> dict:
     return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
 
 
-def run_gpu(xd: dict, gated: bool, out=None):
-    """One call of the CUDA path on device tensors (the pool is updated in place)."""
+def run_gpu(xd: dict, gated: bool, out=None, state_layout="kv"):
+    """One call of the CUDA path on device tensors (the pool is updated in place).
+    With state_layout "vk" the pool in ``xd`` is [pool, H_v, D_v, D_k]."""
     from gated_delta_rule_recurrent_b200 import decode, decode_gated
 
     if gated:
         return decode_gated(xd["query"], xd["key"], xd["value"], xd["a"], xd["b"], xd["dt_bias"],
                             xd["decay_scale"], xd["state_pool"], xd["actual_seq_lengths"],
                             xd["ssm_state_indices"], xd["gk"], xd["num_accepted_tokens"],
-                            xd["scale_value"], out=out)
+                            xd["scale_value"], out=out, state_layout=state_layout)
     return decode(xd["query"], xd["key"], xd["value"], xd["beta"], xd["state_pool"],
                   xd["actual_seq_lengths"], xd["ssm_state_indices"], xd["g"], xd["gk"],
-                  xd["num_accepted_tokens"], xd["scale_value"], out=out)
+                  xd["num_accepted_tokens"], xd["scale_value"], out=out,
+                  state_layout=state_layout)
+
+
+def to_vk(pool: torch.Tensor) -> torch.Tensor:
+    """A [pool, H_v, D_k, D_v] state pool as [pool, H_v, D_v, D_k] (and back)."""
+    return pool.transpose(2, 3).contiguous()
 
 
 def assert_close(got: np.ndarray, ref: np.ndarray, what: str) -> None:

@@ -49,7 +49,7 @@ def test_status_strings_and_version(built_library):
     from gated_delta_rule_recurrent_b200 import binding
 
     L = binding.lib()
-    assert L.gdr_abi_version() == 2
+    assert L.gdr_abi_version() == 3
     for code, name in binding.STATUS_NAMES.items():
         assert L.gdr_status_string(code).decode() == name
     assert L.gdr_status_string(99).decode() == "unknown status"
@@ -71,7 +71,7 @@ def _call_decode(lib, dims, ptr=16, misalign=0, nulls=()):
                           ctypes.c_float(1.0), ctypes.c_void_p(ptr + misalign), None)
 
 
-GOOD = (2, 2, 4, 4, 64, 64, 2)  # B, T, H_qk, H_v, D_k, D_v, pool
+GOOD = (2, 2, 4, 4, 64, 64, 2)  # B, T, H_qk, H_v, D_k, D_v, pool (layout 0)
 
 
 @no_device
@@ -85,6 +85,8 @@ GOOD = (2, 2, 4, 4, 64, 64, 2)  # B, T, H_qk, H_v, D_k, D_v, pool
     ((2, 2, 4, 4, 96, 64, 2), GDR_ERR_UNSUPPORTED),  # D_k not 64/128
     ((2, 2, 4, 4, 64, 96, 2), GDR_ERR_UNSUPPORTED),  # D_v not a multiple of 64
     ((2**30, 1, 1, 64, 64, 512, 2), GDR_ERR_DIMS),    # grid overflow
+    ((2, 2, 4, 4, 64, 64, 2, 2), GDR_ERR_DIMS),      # unknown state layout
+    ((2, 2, 4, 4, 64, 64, 2, -1), GDR_ERR_DIMS),
 ])
 def test_bad_sizes_rejected(built_library, dims, status):
     from gated_delta_rule_recurrent_b200 import binding
