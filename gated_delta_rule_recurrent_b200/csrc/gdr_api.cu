@@ -388,8 +388,8 @@ int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, bool vk, cudaStrea
 
 gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gdr_bf16* key,
                               const gdr_bf16* value, gdr_bf16* state_pool,
-                              const int32_t* asl, const int32_t* idx, const float* gk,
-                              float scale, gdr_bf16* out) {
+                              const int32_t* asl, const int32_t* idx, const int32_t* nat,
+                              const float* gk, float scale, gdr_bf16* out) {
   gdr::DecodeParams p{};
   p.query = query;
   p.key = key;
@@ -399,6 +399,7 @@ gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gd
   p.out = out;
   p.seq_lengths = asl;
   p.state_indices = idx;
+  p.num_accepted = nat;
   p.scale = scale;
   p.B = d->B;
   p.T = d->T;
@@ -475,7 +476,6 @@ GDR_API int gdr_decode(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf
                        const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
                        const float* g, const float* gk, const int32_t* num_accepted_tokens,
                        float scale_value, gdr_bf16* out, gdr_stream_t stream) {
-  (void)num_accepted_tokens;  // does not enter the arithmetic
   int rc = check_dims(dims);
   if (rc != GDR_OK) return rc;
   if (dims->B == 0) return GDR_OK;
@@ -484,7 +484,8 @@ GDR_API int gdr_decode(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf
   if (rc != GDR_OK) return rc;
   if (!beta || !g) return fail(GDR_ERR_NULL, "beta and g must not be NULL");
   gdr::DecodeParams p = base_params(dims, query, key, value, state_pool, actual_seq_lengths,
-                                    ssm_state_indices, gk, scale_value, out);
+                                    ssm_state_indices, num_accepted_tokens, gk, scale_value,
+                                    out);
   p.beta = beta;
   p.g = g;
   return dispatch(p, dims->D_k, false, dims->layout == GDR_LAYOUT_VK,
@@ -497,7 +498,6 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
                            const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
                            const float* gk, const int32_t* num_accepted_tokens,
                            float scale_value, gdr_bf16* out, gdr_stream_t stream) {
-  (void)num_accepted_tokens;
   int rc = check_dims(dims);
   if (rc != GDR_OK) return rc;
   if (dims->B == 0) return GDR_OK;
@@ -507,7 +507,8 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
   if (!a || !b || !dt_bias || !decay_scale)
     return fail(GDR_ERR_NULL, "a, b, dt_bias and decay_scale must not be NULL");
   gdr::DecodeParams p = base_params(dims, query, key, value, state_pool, actual_seq_lengths,
-                                    ssm_state_indices, gk, scale_value, out);
+                                    ssm_state_indices, num_accepted_tokens, gk, scale_value,
+                                    out);
   p.gate_a = a;
   p.gate_b = b;
   p.dt_bias = dt_bias;

@@ -30,6 +30,7 @@ struct DecodeParams {
   uint16_t* out;                // [B, H_v, T, D_v] bf16
   const int32_t* seq_lengths;   // [B]
   const int32_t* state_indices; // [B]
+  const int32_t* num_accepted;  // [B] or NULL: tokens whose state update is committed
   float scale;
   int B, T, H_qk, H_v, D_v, pool_size;
   int group;  // H_v / H_qk

@@ -134,7 +134,7 @@ __host__ __device__ inline ChunkLayout chunk_layout(int T) {
   s.bm = s.a + 256;                      // fp32 [8][8]   B_ts at [t][s], s <= t
   s.beta = s.bm + 256;                   // fp32 [8]
   s.raw = s.beta + 32;                   // u32 [8] g or a words, [8] beta or b words, dt_bias, decay_scale
-  s.meta = s.raw + 80;                   // int32 [4]      length, slot
+  s.meta = s.raw + 80;                   // int32 [4]      length, slot, committed tokens
   s.bytes = (s.meta + 16 + 15) & ~15;
   return s;
 }
@@ -243,7 +243,7 @@ __device__ __forceinline__ int solver_group(int j) { return (j & 1) * 2 + (j >> 
 // adds the slots in warp order.
 template <int DK, int NF, int LC>
 __device__ __forceinline__ void chunk_finalize(uint8_t* vb, const ChunkLayout& lay, float g_lane,
-                                               float scale, int lane, int fw) {
+                                               float scale, int lane, int fw, int n) {
   constexpr int NM = pow2_at_least(LC * LC);  // partial sums, padded for the reduce-scatter
   float g[LC];
 #pragma unroll
@@ -267,25 +267,31 @@ __device__ __forceinline__ void chunk_finalize(uint8_t* vb, const ChunkLayout& l
       kf[t] = bf16_bits_to_f32(sk[t * DK + i]);
       qf[t] = bf16_bits_to_f32(sq[t * DK + i]) * scale;
     }
-    float P = 1.0f;
+    // The committed state is the one after token n - 1 (n = L unless the
+    // call commits fewer tokens): c = P_{n-1}, e_s = P_{s->n-1} k_s for s < n
+    // and 0 for s >= n.
+    float P = 1.0f, c = 0.0f;
 #pragma unroll
     for (int t = 0; t < LC; ++t) {
       P = t == 0 ? d[0] : P * d[t];
       su[t * DK + i] = P * kf[t];  // u_t over the gk entry just read
       sw[t * DK + i] = P * qf[t];
+      if (t == n - 1) c = P;
     }
-    sc[i] = P;
+    sc[i] = c;
 #pragma unroll
     for (int s = 0; s < LC; ++s) {
       float z = kf[s];  // P_{s->t} k_s by running products
+      float e = s == n - 1 ? z : 0.0f;
       mp[s * LC + s] = fmaf(z, qf[s], mp[s * LC + s]);
 #pragma unroll
       for (int t = s + 1; t < LC; ++t) {
         z *= d[t];
         mp[s * LC + t] = fmaf(z, kf[t], mp[s * LC + t]);
         mp[t * LC + s] = fmaf(z, qf[t], mp[t * LC + s]);
+        if (t == n - 1) e = z;
       }
-      se[s * DK + i] = z;
+      se[s * DK + i] = e;
     }
   }
   reduce_scatter<NM>(mp, lane);
@@ -322,17 +328,18 @@ __device__ __forceinline__ void chunk_sum_parts(uint8_t* vb, const ChunkLayout& 
 }
 
 template <int DK, int NF>
-__device__ __forceinline__ void chunk_finalize_any(int L, uint8_t* vb, const ChunkLayout& lay,
-                                                   float g_lane, float scale, int lane, int fw) {
+__device__ __forceinline__ void chunk_finalize_any(int L, int n, uint8_t* vb,
+                                                   const ChunkLayout& lay, float g_lane,
+                                                   float scale, int lane, int fw) {
   switch (L) {
-    case 1: chunk_finalize<DK, NF, 1>(vb, lay, g_lane, scale, lane, fw); break;
-    case 2: chunk_finalize<DK, NF, 2>(vb, lay, g_lane, scale, lane, fw); break;
-    case 3: chunk_finalize<DK, NF, 3>(vb, lay, g_lane, scale, lane, fw); break;
-    case 4: chunk_finalize<DK, NF, 4>(vb, lay, g_lane, scale, lane, fw); break;
-    case 5: chunk_finalize<DK, NF, 5>(vb, lay, g_lane, scale, lane, fw); break;
-    case 6: chunk_finalize<DK, NF, 6>(vb, lay, g_lane, scale, lane, fw); break;
-    case 7: chunk_finalize<DK, NF, 7>(vb, lay, g_lane, scale, lane, fw); break;
-    case 8: chunk_finalize<DK, NF, 8>(vb, lay, g_lane, scale, lane, fw); break;
+    case 1: chunk_finalize<DK, NF, 1>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 2: chunk_finalize<DK, NF, 2>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 3: chunk_finalize<DK, NF, 3>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 4: chunk_finalize<DK, NF, 4>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 5: chunk_finalize<DK, NF, 5>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 6: chunk_finalize<DK, NF, 6>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 7: chunk_finalize<DK, NF, 7>(vb, lay, g_lane, scale, lane, fw, n); break;
+    case 8: chunk_finalize<DK, NF, 8>(vb, lay, g_lane, scale, lane, fw, n); break;
     default: break;
   }
 }
@@ -411,7 +418,8 @@ __device__ __forceinline__ void chunk_sums(const uint8_t* st, const float* su, c
 template <int DK, int VS, int LC>
 __device__ __forceinline__ void chunk_consume(const uint8_t* st, const uint8_t* vb,
                                               const ChunkLayout& lay, int c0, int rg, int lane,
-                                              uint16_t* dst, uint16_t* out_t0, int D_v) {
+                                              uint16_t* dst, uint16_t* out_t0, int D_v,
+                                              bool commit) {
   const float* su = reinterpret_cast<const float*>(vb + lay.u);
   const float* sw = reinterpret_cast<const float*>(vb + lay.w);
   const float* se = reinterpret_cast<const float*>(vb + lay.e);
@@ -455,6 +463,7 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const uint8_t* 
     }
 
   // ---- pass 2: S_L = c o S_0 + sum_s e_s delta_s^T, bf16 once, to the slot
+  if (!commit) return;
   int off[4];
   quad_offsets<DK>(rg, c0, off);
   const uint8_t* st_m = st;
@@ -512,7 +521,7 @@ __device__ __forceinline__ void chunk_consume(const uint8_t* st, const uint8_t* 
 template <int DK, int VS, int LC>
 __device__ __forceinline__ void chunk_consume_vk(const uint8_t* st, const uint8_t* vb,
                                                  const ChunkLayout& lay, int tj, uint16_t* dst,
-                                                 uint16_t* out_t0, int D_v) {
+                                                 uint16_t* out_t0, int D_v, bool commit) {
   constexpr int R = kVkRowsPerThread;
   constexpr int RS = VS / R;  // row stride between a thread's rows
   const float* su = reinterpret_cast<const float*>(vb + lay.u);
@@ -612,6 +621,7 @@ __device__ __forceinline__ void chunk_consume_vk(const uint8_t* st, const uint8_
   }
 
   // ---- pass 2: S_L = c o S_0 + sum_s e_s delta_s^T, bf16 once, to the slot
+  if (!commit) return;
 #pragma unroll 1
   for (int c8 = 0; c8 < DK / 8; ++c8) {
     const ulonglong2 c01 = *reinterpret_cast<const ulonglong2*>(sc + 8 * c8);
@@ -650,16 +660,17 @@ __device__ __forceinline__ void chunk_consume_vk(const uint8_t* st, const uint8_
 template <int DK, int VS>
 __device__ __forceinline__ void chunk_consume_vk_any(int L, const uint8_t* st, const uint8_t* vb,
                                                      const ChunkLayout& lay, int tj,
-                                                     uint16_t* dst, uint16_t* out_t0, int D_v) {
+                                                     uint16_t* dst, uint16_t* out_t0, int D_v,
+                                                     bool commit) {
   switch (L) {
-    case 1: chunk_consume_vk<DK, VS, 1>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 2: chunk_consume_vk<DK, VS, 2>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 3: chunk_consume_vk<DK, VS, 3>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 4: chunk_consume_vk<DK, VS, 4>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 5: chunk_consume_vk<DK, VS, 5>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 6: chunk_consume_vk<DK, VS, 6>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 7: chunk_consume_vk<DK, VS, 7>(st, vb, lay, tj, dst, out_t0, D_v); break;
-    case 8: chunk_consume_vk<DK, VS, 8>(st, vb, lay, tj, dst, out_t0, D_v); break;
+    case 1: chunk_consume_vk<DK, VS, 1>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 2: chunk_consume_vk<DK, VS, 2>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 3: chunk_consume_vk<DK, VS, 3>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 4: chunk_consume_vk<DK, VS, 4>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 5: chunk_consume_vk<DK, VS, 5>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 6: chunk_consume_vk<DK, VS, 6>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 7: chunk_consume_vk<DK, VS, 7>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
+    case 8: chunk_consume_vk<DK, VS, 8>(st, vb, lay, tj, dst, out_t0, D_v, commit); break;
     default: break;
   }
 }
@@ -667,16 +678,17 @@ __device__ __forceinline__ void chunk_consume_vk_any(int L, const uint8_t* st, c
 template <int DK, int VS>
 __device__ __forceinline__ void chunk_consume_any(int L, const uint8_t* st, const uint8_t* vb,
                                                   const ChunkLayout& lay, int c0, int rg, int lane,
-                                                  uint16_t* dst, uint16_t* out_t0, int D_v) {
+                                                  uint16_t* dst, uint16_t* out_t0, int D_v,
+                                                  bool commit) {
   switch (L) {
-    case 1: chunk_consume<DK, VS, 1>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 2: chunk_consume<DK, VS, 2>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 3: chunk_consume<DK, VS, 3>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 4: chunk_consume<DK, VS, 4>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 5: chunk_consume<DK, VS, 5>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 6: chunk_consume<DK, VS, 6>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 7: chunk_consume<DK, VS, 7>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
-    case 8: chunk_consume<DK, VS, 8>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v); break;
+    case 1: chunk_consume<DK, VS, 1>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 2: chunk_consume<DK, VS, 2>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 3: chunk_consume<DK, VS, 3>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 4: chunk_consume<DK, VS, 4>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 5: chunk_consume<DK, VS, 5>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 6: chunk_consume<DK, VS, 6>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 7: chunk_consume<DK, VS, 7>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
+    case 8: chunk_consume<DK, VS, 8>(st, vb, lay, c0, rg, lane, dst, out_t0, D_v, commit); break;
     default: break;
   }
 }
@@ -743,6 +755,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       if (!mbar_wait_bounded(vec0 + 8 * stage, (j / n_stages) & 1)) flag_error(kErrProducerWait);
       int L = reinterpret_cast<const int*>(vb + lay.meta)[0];
       L = L < 0 ? 0 : (L > T ? T : L);
+      const int n_commit = reinterpret_cast<const int*>(vb + lay.meta)[2];
       if (L > 0) {
         float gt = 0.0f;
         if (lane < L) {  // the gate of token `lane`
@@ -761,7 +774,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
           }
           if (fw == 0) reinterpret_cast<float*>(vb + lay.beta)[lane] = bt;
         }
-        chunk_finalize_any<DK, NF>(L, vb, lay, gt, p.scale, lane, fw);
+        chunk_finalize_any<DK, NF>(L, n_commit, vb, lay, gt, p.scale, lane, fw);
       }
       named_barrier(1, 32 * NF);  // every finaliser takes the same path: no early exits
       if (L > 0) chunk_sum_parts<NF>(vb, lay, L, lane, fw);
@@ -775,25 +788,29 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
   if (warp == producer) {
     // ================================================================ producer
     bool failed = false;
-    // lane i holds the slot and length of tile (j & ~31) + i; the next 32
-    // tiles' are loaded 32 tiles ahead
-    auto load_index = [&](int jj, int& slot, int& len) {
+    // lane i holds the slot, length and committed count of tile (j & ~31) + i;
+    // the next 32 tiles' are loaded 32 tiles ahead (no committed-count array:
+    // every token is committed)
+    auto load_index = [&](int jj, int& slot, int& len, int& acc) {
       slot = 0;
       len = 0;
+      acc = 0;
       if (jj < n_mine) {
         const int bb = (blockIdx.x + jj * gridDim.x) / (n_slices * p.H_v);
         slot = p.state_indices[bb];
         len = p.seq_lengths[bb];
+        acc = p.num_accepted != nullptr ? p.num_accepted[bb] : T;
       }
     };
-    int cur_s, cur_L, nxt_s, nxt_L;
-    load_index(lane, cur_s, cur_L);
-    load_index(32 + lane, nxt_s, nxt_L);
+    int cur_s, cur_L, cur_n, nxt_s, nxt_L, nxt_n;
+    load_index(lane, cur_s, cur_L, cur_n);
+    load_index(32 + lane, nxt_s, nxt_L, nxt_n);
     for (int j = 0; j < n_mine; ++j) {
       if (j > 0 && (j & 31) == 0) {
         cur_s = nxt_s;
         cur_L = nxt_L;
-        load_index(j + 32 + lane, nxt_s, nxt_L);
+        cur_n = nxt_n;
+        load_index(j + 32 + lane, nxt_s, nxt_L, nxt_n);
       }
       const int tile = blockIdx.x + j * gridDim.x;
       const int slice = tile % n_slices;
@@ -803,6 +820,8 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       int L = __shfl_sync(0xffffffffu, cur_L, j & 31);
       L = L < 0 ? 0 : (L > T ? T : L);
       if (s < 0 || s >= p.pool_size) L = 0;
+      int n_commit = __shfl_sync(0xffffffffu, cur_n, j & 31);
+      n_commit = n_commit < 0 ? 0 : (n_commit > L ? L : n_commit);
       const int stage = j % n_stages;
       const uint32_t phase = (j / n_stages) & 1;
       uint8_t* vb = vec_base + stage * lay.bytes;
@@ -819,6 +838,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
         int* meta = reinterpret_cast<int*>(vb + lay.meta);
         meta[0] = L;
         meta[1] = s;
+        meta[2] = n_commit;
         if (L > 0) {
           // the L valid tokens' rows are contiguous in HBM: one copy each
           mbar_expect_tx(vbar, L * (DK * 8 + VS * 2));
@@ -899,6 +919,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     L = L < 0 ? 0 : (L > T ? T : L);
     const int s = meta[1];
     if (s < 0 || s >= p.pool_size) L = 0;
+    const bool commit = meta[2] > 0;  // else the slot keeps its bits (pass 2 is skipped)
 
     // out[b, h, t, slice * VS + column]; padded tokens get +0.0
     const size_t bh = static_cast<size_t>(b) * p.H_v + h;
@@ -916,11 +937,11 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       if constexpr (VK) {
         uint16_t* dst =
             p.state_pool + ((static_cast<size_t>(s) * p.H_v + h) * p.D_v + slice * VS) * DK;
-        chunk_consume_vk_any<DK, VS>(L, st, vb, lay, tj, dst, out_t0, p.D_v);
+        chunk_consume_vk_any<DK, VS>(L, st, vb, lay, tj, dst, out_t0, p.D_v, commit);
       } else {
         uint16_t* dst = p.state_pool + (static_cast<size_t>(s) * p.H_v + h) * DK * p.D_v +
                         slice * VS + c0;
-        chunk_consume_any<DK, VS>(L, st, vb, lay, c0, rg, lane, dst, out_t0, p.D_v);
+        chunk_consume_any<DK, VS>(L, st, vb, lay, c0, rg, lane, dst, out_t0, p.D_v, commit);
       }
     }
     __syncwarp();

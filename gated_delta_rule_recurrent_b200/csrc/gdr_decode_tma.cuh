@@ -126,7 +126,7 @@ __host__ __device__ inline StageLayout stage_layout(int T) {
   s.raw = s.rv + T * TS * 16;           // u32 [2][8]  gate scalar words
   s.beta = s.raw + 64;                  // fp32 [8]
   s.kq = s.beta + 32;                   // fp32 [8]       k . (q * scale)
-  s.meta = s.kq + 32;                   // int32 [4]      length, slot
+  s.meta = s.kq + 32;                   // int32 [4]      length, slot, committed tokens
   s.bytes = (s.meta + 16 + 1023) & ~1023;
   return s;
 }
@@ -189,12 +189,14 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     // ================================================================ producer
     constexpr int E = DK / 32;  // row elements per lane in the finalise step
     bool failed = false;
-    // slot and length of the next tile to issue, loaded one iteration ahead
-    int nx_s = 0, nx_L = 0;
+    // slot, length and committed count of the next tile to issue, loaded one
+    // iteration ahead (no committed-count array: all tokens are committed)
+    int nx_s = 0, nx_L = 0, nx_n = 0;
     if (n_mine > 0) {
       const int b0 = blockIdx.x / (p.H_v * n_slices);
       nx_s = p.state_indices[b0];
       nx_L = p.seq_lengths[b0];
+      nx_n = p.num_accepted != nullptr ? p.num_accepted[b0] : T;
     }
     for (int j = 0; j < n_mine + kLookahead; ++j) {
       if (j < n_mine) {
@@ -207,10 +209,12 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         int L = nx_L;
         L = L < 0 ? 0 : (L > T ? T : L);
         if (s < 0 || s >= p.pool_size) L = 0;
+        const int n_commit = nx_n < 0 ? 0 : (nx_n > L ? L : nx_n);
         if (j + 1 < n_mine) {
           const int bn = (tile + gridDim.x) / (n_slices * p.H_v);
           nx_s = p.state_indices[bn];
           nx_L = p.seq_lengths[bn];
+          nx_n = p.num_accepted != nullptr ? p.num_accepted[bn] : T;
         }
         const int stage = j % n_stages;
         const uint32_t phase = (j / n_stages) & 1;
@@ -229,6 +233,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
           int* meta = reinterpret_cast<int*>(st + lay.meta);
           meta[0] = L;
           meta[1] = s;
+          meta[2] = n_commit;
           if (L > 0) {
             mbar_expect_tx(rawb, Shape::kStateBytes + L * (VS * 2 + DK * 8));
             tma_load_3d(smem_addr(st), &pool_map, 0, (s * p.H_v + h) * DK, col0 / 64, rawb);
@@ -380,6 +385,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     L = L > 1 ? 1 : L;  // single-token calls
     const int s = meta[1];
     if (s < 0 || s >= p.pool_size) L = 0;
+    const bool commit = meta[2] > 0;  // else the call leaves the slot's bits as they are
 
     // out[b, h, :, slice * VS + cband : + WCOLS]; padded tokens get +0.0.
     uint16_t* out_band =
@@ -533,9 +539,10 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
             const float2 n2 = upk(fma2(pk(bf16_lo(w.z), bf16_hi(w.z)), d2, mul2(k2, dl2[2])));
             const float2 n3 = upk(fma2(pk(bf16_lo(w.w), bf16_hi(w.w)), d2, mul2(k2, dl2[3])));
             // bf16 round-to-nearest-even, once per call, straight to the slot
-            __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r * RL + rp) * p.D_v),
-                   make_uint4(pack_bf16x2(n0.x, n0.y), pack_bf16x2(n1.x, n1.y),
-                              pack_bf16x2(n2.x, n2.y), pack_bf16x2(n3.x, n3.y)));
+            if (commit)
+              __stcs(reinterpret_cast<uint4*>(dst + static_cast<size_t>(r * RL + rp) * p.D_v),
+                     make_uint4(pack_bf16x2(n0.x, n0.y), pack_bf16x2(n1.x, n1.y),
+                                pack_bf16x2(n2.x, n2.y), pack_bf16x2(n3.x, n3.y)));
           }
         }
       }

@@ -120,8 +120,12 @@ typedef enum gdr_status {
  *   ssm_state_indices   [B] int32, pool slot per item
  *   g                   [B, H_v, T]       fp32
  *   gk                  [B, H_v, T, D_k]  fp32
- *   num_accepted_tokens [B] int32 or NULL: accepted for the page's signature;
- *                       it does not enter the arithmetic and is not read
+ *   num_accepted_tokens [B] int32 or NULL: n = clamp(num_accepted_tokens[b], 0, L)
+ *                       leading tokens of item b are committed. Outputs of all L
+ *                       valid tokens are computed; the slot receives the state
+ *                       after token n - 1 and keeps its bits when n = 0. NULL
+ *                       commits all L (the page gives only the purpose,
+ *                       speculative decoding; this is the library's reading)
  *   scale_value         the page's query scale (1.0 is its default)
  *   out                 [B, H_v, T, D_v]  bf16, fully written
  *   stream              CUDA stream the work is queued on

@@ -31,7 +31,12 @@ in the design notes of the repository):
 * C  exp(g) is a scalar per (b, h, t); exp(gk) scales row i (the D_k axis).
 * D  the state stays in high precision across the tokens of one call and is
      rounded to bfloat16 once, at the end; ``out`` is rounded per token.
-* E  ``num_accepted_tokens`` does not change the arithmetic.
+* E  ``num_accepted_tokens`` (the page gives only its purpose, speculative
+     decoding) selects which state is kept: n = clamp(nat[b], 0, L) leading
+     tokens are committed. Outputs of all L tokens come from the full
+     recurrence; the slot receives the state after token n - 1, and keeps its
+     bits when n = 0. ``None`` means n = L, as does nat = L, the value every
+     workload uses (so the outputs and pool then equal the plain recurrence).
 * E2 lengths are clamped to [0, T]; an item whose slot index is outside
      [0, pool) is skipped (zero output, no slot touched).
 * G  value head h reads query/key head h // (H_v / H_qk).
@@ -143,8 +148,9 @@ def _check_decode_shapes(query, key, value, state, asl, idx, gk):
 
 
 def _decode(query, key, value, state, asl, idx, gk, scale_value, gate_of,
-            round_state, round_out):
-    """Shared token loop of both entry points; ``gate_of(b, t)`` gives (g[H_v], beta[H_v])."""
+            round_state, round_out, nat=None):
+    """Shared token loop of both entry points; ``gate_of(b, t)`` gives (g[H_v], beta[H_v]).
+    ``nat`` holds the committed token counts (reading E), or None."""
     query = np.asarray(query, dtype=np.float64)
     key = np.asarray(key, dtype=np.float64)
     value = np.asarray(value, dtype=np.float64)
@@ -166,7 +172,9 @@ def _decode(query, key, value, state, asl, idx, gk, scale_value, gate_of,
             continue  # reading E2: zero output, no slot touched
         if L == 0:
             continue  # reading J: no token, state unchanged
+        n = L if nat is None else int(min(max(int(nat[b]), 0), L))  # reading E
         S = state_out[s].copy()  # [H_v, D_k, D_v], float64 across the whole call
+        S_commit = None if n == 0 else S
         for t in range(L):
             g_t, beta_t = gate_of(b, t)  # [H_v], [H_v]
             q_t = query[b, hq, t, :] * scale_value  # [H_v, D_k]; q is scaled first
@@ -181,7 +189,10 @@ def _decode(query, key, value, state, asl, idx, gk, scale_value, gate_of,
             S = S + k_t[:, :, None] * delta[:, None, :]
             # step 4, output: o = S^T q
             out[b, :, t, :] = rnd_out(np.einsum("hij,hi->hj", S, q_t))
-        state_out[s] = bf16_round(S) if round_state else S  # reading D
+            if t == n - 1:
+                S_commit = S  # reading E: the state after the last committed token
+        if S_commit is not None:
+            state_out[s] = bf16_round(S_commit) if round_state else S_commit  # reading D
     return out, state_out
 
 
@@ -208,10 +219,9 @@ def recurrent_gated_delta_rule(query, key, value, beta, state, actual_seq_length
     H_v = np.shape(value)[1]
     if beta.shape != (B, H_v, T) or g.shape != (B, H_v, T):
         raise ValueError("beta and g must be [B, H_v, T]")
-    del num_accepted_tokens  # reading E: does not enter the arithmetic
     return _decode(query, key, value, state, actual_seq_lengths, ssm_state_indices, gk,
                    scale_value, lambda b, t: (g[b, :, t], beta[b, :, t]),
-                   round_state, round_out)
+                   round_state, round_out, num_accepted_tokens)
 
 
 def recurrent_gated_delta_rule_gated(query, key, value, a, b, dt_bias, decay_scale, state,
@@ -232,11 +242,9 @@ def recurrent_gated_delta_rule_gated(query, key, value, a, b, dt_bias, decay_sca
     H_v = np.shape(value)[1]
     if a.shape != (B, T, H_v) or braw.shape != (B, T, H_v):
         raise ValueError("a and b must be [B, T, H_v]")
-    del num_accepted_tokens  # reading E
-
     def gate_of(bi, t):
         decay, beta = linear_attention_gate(a[bi, t], dt_bias, decay_scale, braw[bi, t])
         return decay, beta
 
     return _decode(query, key, value, state, actual_seq_lengths, ssm_state_indices, gk,
-                   scale_value, gate_of, round_state, round_out)
+                   scale_value, gate_of, round_state, round_out, num_accepted_tokens)

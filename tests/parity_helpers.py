@@ -52,7 +52,8 @@ def run_oracle(x: dict, gated: bool, items=None):
         idx_sub = np.array([remap.get(int(s), -1) for s in sel])
     sub = {k: (f64(x[k][torch.from_numpy(items)]) if k in PER_TOKEN else None)
            for k in PER_TOKEN}
-    nat = asl[items]
+    nat_all = x.get("num_accepted_tokens")
+    nat = None if nat_all is None else nat_all.to(torch.int64).numpy()[items]
     if gated:
         out, st = recurrent_gated_delta_rule_gated(
             sub["query"], sub["key"], sub["value"], sub["a"], sub["b"], f64(x["dt_bias"]),

@@ -207,3 +207,33 @@ def test_device_errors_reported_without_launch():
         run_gpu(bad, False)
     torch.cuda.synchronize()
     assert np.array_equal(bits(x["state_pool"]), before)
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+@pytest.mark.parametrize("gated", [False, True])
+def test_committed_token_counts(T, gated):
+    """num_accepted_tokens = n in [0, L] per item: outputs of all L tokens,
+    the slot left with the state after n tokens (untouched when n = 0)."""
+    w = workloads.WORKLOADS[0].replace(name=f"commit{T}", B=24, H_qk=2, H_v=4, T=T, D_k=128,
+                                       D_v=128, pool=32, lengths="uniform", indices="subset",
+                                       seed=600 + T)
+    x = workloads.make_inputs(w)
+    L = x["actual_seq_lengths"]
+    gen = torch.Generator().manual_seed(T)
+    n = (torch.rand(L.shape, generator=gen) * (L + 1).float()).floor().to(torch.int32)
+    n[0], n[1] = 0, L[1]  # nothing committed; everything committed
+    n[2] = 99             # clamped to L
+    x["num_accepted_tokens"] = n
+    _roundtrip(x, gated)
+
+
+def test_committed_counts_absent_means_all():
+    x = workloads.make_inputs(3)
+    x["num_accepted_tokens"] = None
+    xd = to_device(x)
+    pool_before = x["state_pool"].clone()
+    out, pool = run_gpu(xd, False)
+    torch.cuda.synchronize()
+    x2 = dict(x)
+    x2["num_accepted_tokens"] = x["actual_seq_lengths"].clone()
+    check_call(x2, out, pool_before, pool.cpu(), False)

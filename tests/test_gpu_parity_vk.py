@@ -100,3 +100,16 @@ def test_same_results_as_the_default_layout():
     d = (out_kv.float() - out_vk.float()).abs()
     assert float(d.max()) <= 2 * (2.0**-7 * float(out_kv.float().abs().max()) + 1e-3)
     assert pool_kv.shape == to_vk(pool_vk).shape
+
+
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_committed_token_counts(T):
+    w = workloads.WORKLOADS[0].replace(name=f"vkcommit{T}", B=16, T=T, D_k=128, D_v=128,
+                                       pool=20, lengths="uniform", indices="subset",
+                                       seed=700 + T)
+    x = workloads.make_inputs(w)
+    L = x["actual_seq_lengths"]
+    gen = torch.Generator().manual_seed(100 + T)
+    x["num_accepted_tokens"] = (torch.rand(L.shape, generator=gen) * (L + 1).float()).floor().to(torch.int32)
+    x["num_accepted_tokens"][0] = 0
+    _roundtrip_vk(x, False)

@@ -42,6 +42,8 @@ MUTATIONS = [
                            "k_t = key[b, hq, t, :] * scale_value  #")]),
     ("state_rounded_every_token", [(OUTL, OUTL + "\n            S = bf16_round(S)")]),
     ("lengths_ignored", [("L = int(min(max(asl[b], 0), T))", "L = T")]),
+    ("committed_count_ignored", [("if t == n - 1:", "if t == L - 1:")]),
+    ("committed_one_token_late", [("if t == n - 1:", "if t == n:")]),
     ("bad_slot_wraps", [("s = int(idx[b])", "s = int(idx[b]) % P")]),
     ("softplus_no_linear_part", [("return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))",
                                   "return np.log1p(np.exp(-np.abs(x)))")]),

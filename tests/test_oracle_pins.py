@@ -303,3 +303,47 @@ def test_state_rounded_once_per_call():
     _, st_once = _run(c, round_out=False)
     _, st_exact = _run(c, round_out=False, round_state=False)
     np.testing.assert_array_equal(st_once, bf16_round(st_exact))
+
+
+# ------------------------------------------------------- committed tokens (reading E)
+
+def test_committed_state_equals_a_shorter_call():
+    """num_accepted_tokens = n < L: the slot receives the state a call over the
+    first n tokens alone leaves (the shorter call is a separate run of the
+    plain recurrence), while every output matches the full-length call."""
+    c = _rand_case(21, B=3, T=5, P=4)
+    full_out, _ = _run(c, round_out=False, round_state=False)
+    n = np.array([2, 5, 1])
+    cn = dict(c, num_accepted_tokens=n)
+    out_n, st_n = _run(cn, round_out=False, round_state=False)
+    np.testing.assert_array_equal(out_n, full_out)
+    short = dict(c, actual_seq_lengths=n, num_accepted_tokens=n)
+    _, st_short = _run(short, round_out=False, round_state=False)
+    np.testing.assert_allclose(st_n, st_short, rtol=1e-13, atol=1e-15)
+    # the committed state differs from the full call's where n < L
+    _, st_full = _run(c, round_out=False, round_state=False)
+    s0 = c["ssm_state_indices"][0]
+    assert np.abs(st_n[s0] - st_full[s0]).max() > 1e-3
+
+
+def test_nothing_committed_keeps_the_slot_bits():
+    c = _rand_case(22, B=2, T=3, P=3)
+    c["state"] = bf16_round(c["state"])
+    n = np.array([0, 0])
+    out0, st0 = _run(dict(c, num_accepted_tokens=n))
+    out_full, _ = _run(c)
+    np.testing.assert_array_equal(out0, out_full)
+    np.testing.assert_array_equal(st0.view(np.int64), c["state"].view(np.int64))
+
+
+def test_committed_count_is_clamped_and_none_means_all():
+    c = _rand_case(23, B=2, T=4, P=2)
+    ref = _run(c)
+    for n in (np.array([9, 4]), np.array([4, 100])):
+        got = _run(dict(c, num_accepted_tokens=n))
+        np.testing.assert_array_equal(got[0], ref[0])
+        np.testing.assert_array_equal(got[1], ref[1])
+    got = _run(dict(c, num_accepted_tokens=None))
+    np.testing.assert_array_equal(got[1], ref[1])
+    neg = _run(dict(c, num_accepted_tokens=np.array([-2, 0])))
+    np.testing.assert_array_equal(neg[1], _run(dict(c, num_accepted_tokens=np.array([0, 0])))[1])
