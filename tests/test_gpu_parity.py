@@ -237,3 +237,40 @@ def test_committed_counts_absent_means_all():
     x2 = dict(x)
     x2["num_accepted_tokens"] = x["actual_seq_lengths"].clone()
     check_call(x2, out, pool_before, pool.cpu(), False)
+
+
+def test_cuda_graph_capture_and_replay():
+    """A decode call captured in a CUDA graph replays with the same results as
+    a direct call: the library queues only kernels on the caller's stream
+    (configuration and tensor maps are host work done at capture time)."""
+    from gated_delta_rule_recurrent_b200 import decode
+
+    x = workloads.make_inputs(3)
+    direct = to_device(x)
+    out_ref, pool_ref = run_gpu(direct, False)
+    torch.cuda.synchronize()
+    xd = to_device(x)
+    pool0 = xd["state_pool"].clone()
+    out = torch.empty_like(out_ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up outside the graph (first-call setup)
+        run_gpu(xd, False, out=out)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    xd["state_pool"].copy_(pool0)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        decode(xd["query"], xd["key"], xd["value"], xd["beta"], xd["state_pool"],
+               xd["actual_seq_lengths"], xd["ssm_state_indices"], xd["g"], xd["gk"],
+               xd["num_accepted_tokens"], xd["scale_value"], out=out)
+    xd["state_pool"].copy_(pool0)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(out.cpu()), bits(out_ref.cpu()))
+    assert np.array_equal(bits(xd["state_pool"].cpu()), bits(pool_ref.cpu()))
+    # a second replay continues from the pool the first one left
+    g.replay()
+    torch.cuda.synchronize()
+    assert not np.array_equal(bits(xd["state_pool"].cpu()), bits(pool_ref.cpu()))
