@@ -166,9 +166,13 @@ def decode(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, beta: to
 
     Argument order and defaults follow the op's page. ``state_pool`` is
     updated in place and returned as the second result (the page's
-    ``state_out``). ``state_layout`` "vk" takes the pool as [pool, H_v, D_v,
-    D_k] (k contiguous) instead of the page's [pool, H_v, D_k, D_v]. Queued on
-    the current CUDA stream; no synchronisation.
+    ``state_out``). ``num_accepted_tokens`` (optional, [B] int32) is the
+    number of leading tokens whose state update is committed: outputs of all
+    valid tokens are computed, the slot keeps the state after the first n
+    (unchanged for n = 0); None commits them all. ``state_layout`` "vk" takes
+    the pool as [pool, H_v, D_v, D_k] (k contiguous) instead of the page's
+    [pool, H_v, D_k, D_v]. Queued on the current CUDA stream; no
+    synchronisation.
     """
     device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
                                         ssm_state_indices, gk, num_accepted_tokens, out,

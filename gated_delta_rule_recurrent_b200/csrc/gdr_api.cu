@@ -1,5 +1,6 @@
 // C ABI of libgdr (declared in include/gdr.h): host-side argument checks and
-// kernel dispatch for the recurrent gated-delta-rule decode step.
+// kernel dispatch for the recurrent gated-delta-rule decode step and the
+// standalone LinearAttentionGate op.
 //
 // Everything here runs on the host before any launch. A failed check returns
 // its status with nothing queued; device values (lengths, slot indices) are
@@ -31,7 +32,7 @@ int fail(int status, const std::string& what) {
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
-// Checks shared by both entry points. Returns GDR_OK or a failure status.
+// Checks shared by both decode entry points. Returns GDR_OK or a failure status.
 int check_dims(const gdr_dims* d) {
   if (d == nullptr) return fail(GDR_ERR_NULL, "dims is NULL");
   if (d->B < 0) return fail(GDR_ERR_DIMS, "B must be >= 0");

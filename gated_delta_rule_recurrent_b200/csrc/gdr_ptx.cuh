@@ -11,7 +11,9 @@
 
 namespace gdr {
 
-// Bits of the device error word.
+// Bits of the device error word: a consumer's wait for a ready tile; a wait on
+// the producing side (a free stage, or landed copies to finalise); the final
+// wait for copies still in flight.
 constexpr unsigned kErrConsumerWait = 1u;
 constexpr unsigned kErrProducerWait = 2u;
 constexpr unsigned kErrDrainWait = 4u;
@@ -19,7 +21,6 @@ constexpr unsigned kErrDrainWait = 4u;
 static __device__ unsigned int g_device_error = 0;
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
-
 
 // Byte offset of (row i, 16-byte chunk holding column col) in a state tile
 // loaded by TMA with the 128-byte swizzle as [col / 64][row][64 columns]:
@@ -62,8 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of parity `parity` to complete, for at most
-// kWaitLimitCycles. Returns false when the budget ran out.
 // As mbar_try_wait, but the thread may stay suspended in the instruction for
 // up to `hint_ns` nanoseconds while the phase is incomplete (it resumes as
 // soon as the phase completes), so a waiting warp takes few issue slots.
@@ -82,6 +81,8 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 
 constexpr uint32_t kWaitSuspendNs = 20000;
 
+// Wait for the phase of parity `parity` to complete, for at most
+// kWaitLimitCycles. Returns false when the budget ran out.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -153,13 +154,6 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
   unsigned long long d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-__device__ __forceinline__ void unpack_bf16x8(const uint4 w, float (&f)[8]) {
-  f[0] = bf16_lo(w.x); f[1] = bf16_hi(w.x);
-  f[2] = bf16_lo(w.y); f[3] = bf16_hi(w.y);
-  f[4] = bf16_lo(w.z); f[5] = bf16_hi(w.z);
-  f[6] = bf16_lo(w.w); f[7] = bf16_hi(w.w);
 }
 
 // Named barrier over `count` threads (a multiple of 32) of the CTA.

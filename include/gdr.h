@@ -206,9 +206,10 @@ GDR_API const char* gdr_status_string(int status);
 GDR_API const char* gdr_last_error(void);
 
 /* Device-side error word of the current device, OR-ed over every kernel run
- * since the last reset: bit 0 = a consumer wait on staged data ran out of time,
- * bit 1 = the producer's wait for a free stage ran out of time, bit 2 = the
- * final wait for in-flight copies ran out of time. A wait that runs out never
+ * since the last reset: bit 0 = a consumer's wait for a ready tile ran out of
+ * time, bit 1 = a wait on the producing side (a free stage, or landed copies
+ * to prepare) ran out of time, bit 2 = the final wait for in-flight copies ran
+ * out of time. A wait that runs out never
  * hangs the kernel: it flags the word and the kernel finishes, and the outputs
  * of that call are invalid. Writes the word to *flags and clears it when
  * `reset` is nonzero. SYNCHRONISES the device (a blocking copy). No
