@@ -23,7 +23,8 @@ HASH_PATH = LIB_PATH + ".srchash"
 
 SOURCES = [os.path.join(CSRC, "gdr_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, name) for name in (
-    "gdr_decode.cuh", "gdr_ptx.cuh", "gdr_decode_tma.cuh", "gdr_decode_chunk.cuh", "gdr_gate.cuh")] + [
+    "gdr_decode.cuh", "gdr_ptx.cuh", "gdr_decode_tma.cuh", "gdr_decode_chunk.cuh", "gdr_decode_chunk_tc.cuh",
+    "gdr_umma.cuh", "gdr_gate.cuh")] + [
     os.path.join(INCLUDE, "gdr.h")]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -18,6 +18,7 @@
 #include "gdr.h"
 #include "gdr_decode.cuh"
 #include "gdr_decode_chunk.cuh"
+#include "gdr_decode_chunk_tc.cuh"
 #include "gdr_decode_tma.cuh"
 #include "gdr_gate.cuh"
 
@@ -313,6 +314,70 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
   return GDR_OK;
 }
 
+// ---------------------------------------------------------------- tensor-core chunk path (T >= 2, 128 x 128)
+
+// One persistent CTA per SM with kTcGroups consumer groups; each group gets
+// as many stages as shared memory holds (at most 4).
+template <bool GATED>
+int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
+  static ChunkConfig cache[kMaxDevices][gdr::kMaxT + 1];
+  static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
+  if (ready[dev][T].load(std::memory_order_acquire)) {
+    *out = cache[dev][T];
+    return GDR_OK;
+  }
+  auto kernel = gdr::decode_chunk_tc_kernel<GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         props.smem_optin);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
+  constexpr int ng = gdr::kTcGroups;
+  int per = 1;
+  while (per < 4 && gdr::tc_smem_bytes(T, (per + 1) * ng, ng) <= props.smem_optin) ++per;
+  if (gdr::tc_smem_bytes(T, per * ng, ng) > props.smem_optin)
+    return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+  ChunkConfig c;
+  c.n_stages = per * ng;
+  c.smem = gdr::tc_smem_bytes(T, c.n_stages, ng);
+  c.threads = gdr::kTcMaxThreads;
+  int resident = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, c.threads, c.smem);
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("occupancy query: ") + cudaGetErrorString(err));
+  if (resident < 1) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit on an SM");
+  cache[dev][T] = c;
+  ready[dev][T].store(true, std::memory_order_release);
+  *out = c;
+  return GDR_OK;
+}
+
+template <bool GATED>
+int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
+  DeviceProps props;
+  int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  ChunkConfig cfg;
+  rc = chunk_tc_config<GATED>(dev, p.T, props, &cfg);
+  if (rc != GDR_OK) return rc;
+  CUtensorMap map;
+  rc = encode_pool_map(p, gdr::kTcDK, gdr::kTcVS, false, &map);
+  if (rc != GDR_OK) return rc;
+  const int n_tiles = p.B * p.H_v * (p.D_v / gdr::kTcVS);
+  const int grid = n_tiles < props.sms ? n_tiles : props.sms;
+  gdr::decode_chunk_tc_kernel<GATED><<<grid, cfg.threads, cfg.smem, stream>>>(map, p, n_tiles,
+                                                                            cfg.n_stages);
+  err = cudaGetLastError();
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  return GDR_OK;
+}
+
 using LaunchFn = int (*)(const gdr::DecodeParams&, cudaStream_t);
 struct SliceKernel {
   int vs;
@@ -324,8 +389,8 @@ struct SliceKernel {
 // thread count of a block caps the registers ptxas may give a thread (255 up
 // to 256 threads, 168 up to 384, 128 up to 512, 96 up to 640), and a
 // single-token call keeps no state in registers (about 75 of them), so a
-// full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls use
-// the chunked kernel (64 columns per consumer warp).
+// full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls that
+// the tensor-core kernel does not take use the CUDA-core chunked kernel.
 template <bool GATED>
 const SliceKernel* slice_kernels(int D_k, bool one, bool vk, int* n) {
   static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED>},
@@ -356,10 +421,11 @@ const SliceKernel* slice_kernels(int D_k, bool one, bool vk, int* n) {
   return one ? k128_one : k128_many;
 }
 
-// Column-slice width: the widest width that divides D_v and still gives every
-// SM GDR_MIN_TILES_PER_SM tiles, else the narrowest one; a width whose stage
-// ring does not fit in shared memory (long T) falls back to the next narrower
-// one.
+// Multi-token calls with D_k = 128 and 128-column slices take the
+// tensor-core chunked kernel. Otherwise the column-slice width is the widest
+// width that divides D_v and still gives every SM GDR_MIN_TILES_PER_SM tiles,
+// else the narrowest one; a width whose stage ring does not fit in shared
+// memory (long T) falls back to the next narrower one.
 int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, bool vk, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
@@ -368,6 +434,10 @@ int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, bool vk, cudaStrea
   if (rc != GDR_OK) return rc;
   int n = 0;
   const bool one = p.T == 1;
+  if (!one && !vk && D_k == gdr::kTcDK && p.D_v % gdr::kTcVS == 0) {
+    rc = gated ? launch_chunk_tc<true>(p, stream) : launch_chunk_tc<false>(p, stream);
+    if (rc != GDR_ERR_UNSUPPORTED) return rc;
+  }
   const SliceKernel* ks = gated ? slice_kernels<true>(D_k, one, vk, &n)
                                 : slice_kernels<false>(D_k, one, vk, &n);
   int first = -1;

@@ -59,6 +59,8 @@ def test_large_batch_gated_full_size_sampled():
     (128, 64, 7, 7, 1),
     (128, 128, 2, 2, 2),
     (64, 512, 4, 4, 6),
+    (128, 256, 2, 4, 8),    # two 128-column slices, all 8 tokens
+    (128, 512, 1, 3, 3),    # four slices, multi-query
 ])
 @pytest.mark.parametrize("gated", [False, True])
 def test_ragged_shapes(D_k, D_v, H_qk, H_v, T, gated):
