@@ -45,7 +45,9 @@
 //   4. the elected thread issues pass 2 (2 MMAs); each thread then reads its
 //      row of D2, adds c_i S_0[i, :] from the staged tile, rounds to bf16 and
 //      writes the row back over S_0 in place; the elected thread stores the
-//      tile to the slot with one TMA store.
+//      tile to the slot with one TMA store and releases the stage once the
+//      store has read it, after finalising the group's next tile (so the
+//      store's read of the stage overlaps that work).
 // The producer warp starts the copies of each tile as in the chunked kernel
 // (one TMA box for the state, bulk copies for the k, q, gk and v rows of the
 // valid tokens, 4-byte copies for the gate scalars).
@@ -321,27 +323,35 @@ __device__ __forceinline__ void tc_solve_any(int L, const uint32_t (&x)[32], con
 
 // Row i of S_n = c_i S_0[i, :] + D2[i, :], rounded to bf16 and written over
 // S_0 in the staged (swizzled) tile, 32 columns per TMEM read.
+// 64 columns per round: two TMEM reads in flight, and the round's 8 state
+// chunks read from shared memory while they are.
 __device__ __forceinline__ void tc_new_state_row(uint8_t* st, uint32_t d2_lane, float c, int i) {
   const unsigned long long cc = pk(c, c);
 #pragma unroll
-  for (int k = 0; k < kTcVS / 32; ++k) {
-    uint32_t acc[32];
-    tmem_ld32(d2_lane + 32 * k, acc);
+  for (int k = 0; k < kTcVS / 64; ++k) {
+    uint32_t acc[2][32];
+    tmem_ld32(d2_lane + 64 * k, acc[0]);
+    tmem_ld32(d2_lane + 64 * k + 32, acc[1]);
+    uint4* ptr[8];
+    uint4 s0[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      ptr[q] = reinterpret_cast<uint4*>(st + swz_offset<kTcDK>(i, 64 * k + 8 * q));
+      s0[q] = *ptr[q];
+    }
     tmem_wait_ld();
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4* p = reinterpret_cast<uint4*>(st + swz_offset<kTcDK>(i, 32 * k + 8 * q));
-      const uint4 s0 = *p;
-      const uint32_t sw[4] = {s0.x, s0.y, s0.z, s0.w};
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t sw[4] = {s0[q].x, s0[q].y, s0[q].z, s0[q].w};
+      const uint32_t* a = &acc[q >> 2][8 * (q & 3)];
       uint32_t nw[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const unsigned long long a = pk(__uint_as_float(acc[8 * q + 2 * e]),
-                                        __uint_as_float(acc[8 * q + 2 * e + 1]));
-        const float2 r = upk(fma2(cc, pk(bf16_lo(sw[e]), bf16_hi(sw[e])), a));
+        const float2 r = upk(fma2(cc, pk(bf16_lo(sw[e]), bf16_hi(sw[e])),
+                                  pk(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]))));
         nw[e] = pack_bf16x2(r.x, r.y);
       }
-      *p = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+      *ptr[q] = make_uint4(nw[0], nw[1], nw[2], nw[3]);
     }
   }
 }
@@ -519,12 +529,14 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     const uint32_t lane_field = static_cast<uint32_t>(32 * wq) << 16;
     const uint32_t d2 = tmem_base + kTcVS * group;
     const uint32_t d1 = tmem_base + kTcVS * n_groups + kTcN1 * group;
-    const uint32_t b1_addr = smem_addr(gb + kTcB1);
-    const uint32_t e_addr = smem_addr(gb + kTcE);
-    const uint32_t dl_addr = smem_addr(gb + kTcDL);
+    // operand descriptors at K step 0 (the state's depends on the stage)
+    const uint64_t b1_desc = umma_desc(smem_addr(gb + kTcB1), 128, 2048, kUmmaInterleave);
+    const uint64_t e_desc = umma_desc(smem_addr(gb + kTcE), 128, 512, kUmmaInterleave);
+    const uint64_t dl_desc = umma_desc(smem_addr(gb + kTcDL), 128, 512, kUmmaInterleave);
     constexpr uint32_t idesc1 = umma_idesc_bf16<kTcVS, kTcN1, true, true>();
     constexpr uint32_t idesc2 = umma_idesc_bf16<kTcDK, kTcVS, false, false>();
     uint32_t mma_phase = 0;
+    int held = -1;  // the stage whose new state is still being stored (elected thread)
 
     for (int it = group; it < n_mine; it += n_groups) {
       const int tile = blockIdx.x + it * gridDim.x;
@@ -571,6 +583,11 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         c_row = tc_finalize_any(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
       }
       fence_async_smem();
+      if (elected && held >= 0) {  // the previous tile's store has read its stage by now
+        bulk_wait_read_all();
+        mbar_arrive(empty0 + 8 * held);
+        held = -1;
+      }
       ok_self = mbar_wait_bounded(sta0 + 8 * stage, phase) && ok_self;
       if (!ok_self) flag_error(kErrConsumerWait);
       tc_fence_before();
@@ -578,14 +595,17 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
 
       // ---- 2. pass 1 on the tensor cores; A and B on the CUDA cores
       if (L > 0) {
-        if (elected) {
-          tc_fence_after();
-          const uint32_t st_addr = smem_addr(st);
+        if (wq == 0) {  // warp-uniform: one lane issues
+          const uint64_t st_desc = umma_desc(smem_addr(st), DK * 128, 1024, kUmmaSwizzle128);
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < DK / 16; ++ks)
-            umma_bf16(d1, umma_desc(st_addr + ks * 2048, DK * 128, 1024, kUmmaSwizzle128),
-                      umma_desc(b1_addr + ks * 256, 128, 2048, kUmmaInterleave), idesc1, ks > 0);
-          umma_commit(mbar);
+            for (int ks = 0; ks < DK / 16; ++ks)
+              umma_bf16(d1, umma_desc_advance(st_desc, ks * 2048),
+                        umma_desc_advance(b1_desc, ks * 256), idesc1, ks > 0);
+            umma_commit(mbar);
+          }
+          __syncwarp();
         }
         tc_sum_parts(gb, L, r);
       }
@@ -608,13 +628,16 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       // ---- 4. pass 2 and the new state, when any token is committed
       const bool commit = L > 0 && n_commit > 0;  // else the slot keeps its bits
       if (commit) {
-        if (elected) {
-          tc_fence_after();
+        if (wq == 0) {
+          if (elect_one()) {
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < kTcK2 / 16; ++ks)
-            umma_bf16(d2, umma_desc(e_addr + ks * 256, 128, 512, kUmmaInterleave),
-                      umma_desc(dl_addr + ks * 256, 128, 512, kUmmaInterleave), idesc2, ks > 0);
-          umma_commit(mbar);
+            for (int ks = 0; ks < kTcK2 / 16; ++ks)
+              umma_bf16(d2, umma_desc_advance(e_desc, ks * 256),
+                        umma_desc_advance(dl_desc, ks * 256), idesc2, ks > 0);
+            umma_commit(mbar);
+          }
+          __syncwarp();
         }
         if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
         mma_phase ^= 1u;
@@ -624,16 +647,23 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       }
       tc_fence_before();
       named_barrier(bar_id, kTcGroupThreads);  // new state staged; D2 reads done
+      // the store runs while the group finalises its next tile; the stage is
+      // released once the store has read it
       if (elected) {
         if (commit) {
           tma_store_3d(&pool_map, 0, (s * p.H_v + h) * DK, slice * VS / 64, smem_addr(st));
           bulk_commit_group();
-          bulk_wait_read_all();  // the stage may be refilled once the store has read it
         }
-        mbar_arrive(empty0 + 8 * stage);
+        held = stage;
       }
     }
-    if (elected) bulk_wait_all();
+    if (elected) {
+      if (held >= 0) {
+        bulk_wait_read_all();
+        mbar_arrive(empty0 + 8 * held);
+      }
+      bulk_wait_all();
+    }
   }
 
   // every warp arrives here: free the tensor memory once no thread can touch it

@@ -64,6 +64,23 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16() {
 
 // ---------------------------------------------------------------- MMA
 
+// True in exactly one active lane of the warp (all lanes must execute it).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t is_elected;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(is_elected));
+  return is_elected != 0;
+}
+
+// The descriptor `desc` with its start address moved on by `bytes` (a
+// multiple of 16 that keeps the address inside shared memory).
+__host__ __device__ __forceinline__ uint64_t umma_desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // D[M x N] (+)= A[M x 16] * B[N x 16]^T for one instruction (K = 16), issued
 // by one thread; D in TMEM at `d_tmem` (lane 0, first column).
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
