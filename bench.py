@@ -70,6 +70,15 @@ def kernel_source_hash():
     return h.hexdigest()
 
 
+def decode_kernel_name(w, layout):
+    """The kernel the library launches for this workload (one per call)."""
+    if w.T == 1 and layout == "kv":
+        return "gdr::decode_tma_kernel"
+    if layout == "kv" and w.D_k == 128 and w.D_v % 128 == 0:
+        return "gdr::decode_chunk_tc_kernel"
+    return "gdr::decode_chunk_kernel"
+
+
 def recorded_traffic(workload_name, layout):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     this workload and layout with the current kernel source; else None."""
@@ -331,9 +340,12 @@ def run_gdr(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    # Events only at the two ends of the region: the steps run back to back
+    # (the host enqueues a call in ~25 us, ahead of the device), one decode
+    # launch per step, so the average launch duration is the region over the
+    # launches. (An event pair around every launch leaves the device idle for
+    # a few microseconds between launches, which a short step would count.)
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     region0 = torch.cuda.Event(enable_timing=True)
     region1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -341,9 +353,7 @@ def run_gdr(args):
     host_t0 = time.time()
     region0.record(stream)
     for i in range(K):
-        ev[i][0].record(stream)
         step()
-        ev[i][1].record(stream)
     region1.record(stream)
     torch.cuda.synchronize(dev)
     host_t1 = time.time()
@@ -351,8 +361,7 @@ def run_gdr(args):
     launches = K  # one kernel per step (the decode kernel)
     region_ms = max_over_ranks(region0.elapsed_time(region1))
     total_tokens = distributed.sum_over_ranks(n_tokens * K, dev)
-    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-    kernel_ms = max_over_ranks(kernel_ms)
+    kernel_ms = region_ms / launches
     clocks = sampler.summary(host_t0, host_t1)
 
     # ---- end to end through the public API: pinned host inputs copied in and
@@ -409,8 +418,7 @@ def run_gdr(args):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth",
-            "kernel": ("gdr::decode_tma_kernel" if w.T == 1 and args.layout == "kv"
-                       else "gdr::decode_chunk_kernel"), "kernel_ms": kernel_ms,
+            "kernel": decode_kernel_name(w, args.layout), "kernel_ms": kernel_ms,
             "bytes_per_launch": step_bytes, "traffic": recorded_traffic(w.name, args.layout),
         },
         "e2e": e2e,
@@ -497,23 +505,19 @@ def run_gate(args):
         step()
     torch.cuda.synchronize(dev)
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     stream = torch.cuda.current_stream(dev)
     r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     host_t0 = time.time()
     r0.record(stream)
-    for i in range(K):
-        ev[i][0].record(stream)
+    for i in range(K):  # back to back, events at the region's ends only
         step()
-        ev[i][1].record(stream)
     r1.record(stream)
     torch.cuda.synchronize(dev)
     host_t1 = time.time()
     clocks = sampler.summary(host_t0, host_t1)
     sampler.stop()
     region_ms = r0.elapsed_time(r1)
-    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    kernel_ms = region_ms / K  # per step: the vector launch (and the tail launch, if any)
     peak, peak_src = measured_hbm_peak()
     achieved = step_bytes / (kernel_ms * 1e-3) / 1e9
     # the fp64 oracle on a bounded sample of rows, one thread

@@ -245,7 +245,6 @@ struct ChunkConfig {
   int n_stages = 0;
   int smem = 0;
   int threads = 0;
-  int order_cap = 0;  // tensor-core kernel: entries of the CTA's tile order
 };
 
 
@@ -337,14 +336,12 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
     return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
   constexpr int ng = gdr::kTcGroups;
   int per = 1;
-  while (per < 4 && gdr::tc_smem_bytes(T, (per + 1) * ng, ng, 0) <= props.smem_optin) ++per;
-  if (gdr::tc_smem_bytes(T, per * ng, ng, 0) > props.smem_optin)
+  while (per < 4 && gdr::tc_smem_bytes(T, (per + 1) * ng, ng) <= props.smem_optin) ++per;
+  if (gdr::tc_smem_bytes(T, per * ng, ng) > props.smem_optin)
     return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
   ChunkConfig c;
   c.n_stages = per * ng;
-  // the rest of shared memory holds the CTA's tile order
-  c.order_cap = (props.smem_optin - gdr::tc_smem_bytes(T, c.n_stages, ng, 0)) / 4;
-  c.smem = gdr::tc_smem_bytes(T, c.n_stages, ng, c.order_cap);
+  c.smem = gdr::tc_smem_bytes(T, c.n_stages, ng);
   c.threads = gdr::kTcMaxThreads;
   int resident = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, c.threads, c.smem);
@@ -373,8 +370,8 @@ int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
   if (rc != GDR_OK) return rc;
   const int n_tiles = p.B * p.H_v * (p.D_v / gdr::kTcVS);
   const int grid = n_tiles < props.sms ? n_tiles : props.sms;
-  gdr::decode_chunk_tc_kernel<GATED><<<grid, cfg.threads, cfg.smem, stream>>>(
-      map, p, n_tiles, cfg.n_stages, cfg.order_cap);
+  gdr::decode_chunk_tc_kernel<GATED><<<grid, cfg.threads, cfg.smem, stream>>>(map, p, n_tiles,
+                                                                            cfg.n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));

@@ -29,8 +29,8 @@
 // stay on the CUDA cores.
 //
 // CTA: NG consumer groups of 4 warps and one producer warp, one CTA per SM,
-// persistent over its share of the tiles (see tc_tile_order); group g takes
-// every NG-th of them. Thread r of a group (warp w = r / 32, so TMEM lanes 32 (w % 4)
+// persistent over tiles blockIdx.x, + gridDim.x, ...; group g takes every
+// NG-th tile. Thread r of a group (warp w = r / 32, so TMEM lanes 32 (w % 4)
 // + lane) is row i = r of the tile in the row-wise steps and column j = r in
 // the column-wise ones:
 //   1. finalise (row i): decays, u, w, e, c, and its share of A and B (a warp
@@ -119,66 +119,11 @@ constexpr int kTcBm = 25856;    // fp32 [8][8] B_ts at [t][s], s <= t
 constexpr int kTcGroupBytes = 26624;
 
 // Three mbarriers per stage (vectors landed, state landed, stage released)
-// and one per group (its MMAs done), the TMEM address, then `order_cap`
-// entries of the CTA's tile order.
-__host__ __device__ inline int tc_smem_bytes(int T, int n_stages, int n_groups, int order_cap) {
+// and one per group (its MMAs done).
+__host__ __device__ inline int tc_smem_bytes(int T, int n_stages, int n_groups) {
   const int vec = (n_stages * tc_layout(T).bytes + 1023) & ~1023;
   return 1024 /* alignment slack */ + n_stages * kTcStateBytes + vec + n_groups * kTcGroupBytes +
-         (3 * n_stages + n_groups) * 8 + 16 + 4 * order_cap;
-}
-
-// ---------------------------------------------------------------- tile order
-
-// The tiles of a call sorted by the clamped token count of their item, most
-// tokens first (items with equal counts in index order, an item's tiles in
-// tile order), and dealt round-robin: this CTA takes sorted positions
-// blockIdx.x, + gridDim.x, ..., so every CTA gets a near-equal share of the
-// costly tiles. One warp writes order[j] = the tile of this CTA's j-th
-// position, in two passes over the items (a count per token count, then each
-// item's position from ballots).
-__device__ __forceinline__ void tc_tile_order(const DecodeParams& p, int per_item, int* order,
-                                              int lane) {
-  const int T = p.T;
-  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  auto item_len = [&](int b) {
-    int L = p.seq_lengths[b];
-    L = L < 0 ? 0 : (L > T ? T : L);
-    const int s = p.state_indices[b];
-    return (s < 0 || s >= p.pool_size) ? 0 : L;
-  };
-  int count[kMaxT + 1];
-#pragma unroll
-  for (int v = 0; v <= kMaxT; ++v) count[v] = 0;
-  for (int b0 = 0; b0 < p.B; b0 += 32) {
-    const int L = b0 + lane < p.B ? item_len(b0 + lane) : -1;
-#pragma unroll
-    for (int v = 0; v <= kMaxT; ++v) count[v] += __popc(__ballot_sync(0xffffffffu, L == v));
-  }
-  int start[kMaxT + 1];  // first sorted item position of each token count
-  int acc = 0;
-#pragma unroll
-  for (int v = kMaxT; v >= 0; --v) {
-    start[v] = acc;
-    acc += count[v];
-  }
-  const unsigned below = (1u << lane) - 1u;
-  for (int b0 = 0; b0 < p.B; b0 += 32) {
-    const int b = b0 + lane;
-    const int L = b < p.B ? item_len(b) : -1;
-    int pos = 0;
-#pragma unroll
-    for (int v = 0; v <= kMaxT; ++v) {
-      const unsigned m = __ballot_sync(0xffffffffu, L == v);
-      if (L == v) pos = start[v] + __popc(m & below);
-      start[v] += __popc(m);
-    }
-    if (b < p.B) {
-      // this item's sorted tile positions are [R, R + per_item); take those = c mod G
-      const int R = pos * per_item;
-      for (int r = R + ((c - R % G) + G) % G; r < R + per_item; r += G)
-        order[(r - c) / G] = b * per_item + (r - R);
-    }
-  }
+         (3 * n_stages + n_groups) * 8 + 16;
 }
 
 // Eight fp32 values as bf16 (hi, lo) parts, packed in pairs: hi = bf16(x),
@@ -429,7 +374,7 @@ __device__ __forceinline__ uint32_t tc_phase(int j, int n_groups, int per_group)
 template <bool GATED>
 __global__ void __launch_bounds__(kTcMaxThreads, 1)
     decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
-                           const int n_tiles, const int n_stages, const int order_cap) {
+                           const int n_tiles, const int n_stages) {
   constexpr int DK = kTcDK, VS = kTcVS;
   const int T = p.T;
   const TcLayout lay = tc_layout(T);
@@ -447,7 +392,6 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
   const uint32_t empty0 = sta0 + 8 * n_stages;    // the group is done with the stage
   const uint32_t mma0 = empty0 + 8 * n_stages;    // a group's MMAs are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * n_stages + n_groups);
-  int* order = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(tmem_slot) + 16);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -456,11 +400,6 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
   const int n_slices = p.D_v / VS;
   const int n_mine = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                      static_cast<int>(gridDim.x);
-  // this CTA's j-th tile: from the sorted order when it fits in shared memory
-  const bool sorted = n_mine <= order_cap;
-  auto tile_of = [&](int j) {
-    return sorted ? order[j] : static_cast<int>(blockIdx.x) + j * static_cast<int>(gridDim.x);
-  };
 
   if (tid == 0) {
     for (int i = 0; i < n_stages; ++i) {
@@ -476,7 +415,6 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     tmem_alloc(smem_addr(tmem_slot), kTcTmemCols);
     tmem_relinquish();
   }
-  if (warp == producer && sorted) tc_tile_order(p, n_slices * p.H_v, order, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -492,7 +430,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       len = 0;
       acc = 0;
       if (jj < n_mine) {
-        const int bb = tile_of(jj) / (n_slices * p.H_v);
+        const int bb = (blockIdx.x + jj * gridDim.x) / (n_slices * p.H_v);
         slot = p.state_indices[bb];
         len = p.seq_lengths[bb];
         acc = p.num_accepted != nullptr ? p.num_accepted[bb] : T;
@@ -508,7 +446,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         cur_n = nxt_n;
         load_index(j + 32 + lane, nxt_s, nxt_L, nxt_n);
       }
-      const int tile = tile_of(j);
+      const int tile = blockIdx.x + j * gridDim.x;
       const int slice = tile % n_slices;
       const int h = (tile / n_slices) % p.H_v;
       const int b = tile / (n_slices * p.H_v);
@@ -601,7 +539,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     int held = -1;  // the stage whose new state is still being stored (elected thread)
 
     for (int it = group; it < n_mine; it += n_groups) {
-      const int tile = tile_of(it);
+      const int tile = blockIdx.x + it * gridDim.x;
       const int slice = tile % n_slices;
       const int h = (tile / n_slices) % p.H_v;
       const int b = tile / (n_slices * p.H_v);
