@@ -318,7 +318,7 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
 
 // One persistent CTA per SM with kTcGroups consumer groups; each group gets
 // as many stages as shared memory holds (at most 4).
-template <bool GATED>
+template <bool GATED, bool VK>
 int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   static ChunkConfig cache[kMaxDevices][gdr::kMaxT + 1];
   static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
@@ -326,7 +326,7 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
     *out = cache[dev][T];
     return GDR_OK;
   }
-  auto kernel = gdr::decode_chunk_tc_kernel<GATED>;
+  auto kernel = gdr::decode_chunk_tc_kernel<GATED, VK>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          props.smem_optin);
   if (err == cudaSuccess)
@@ -354,7 +354,7 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
   return GDR_OK;
 }
 
-template <bool GATED>
+template <bool GATED, bool VK>
 int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -363,15 +363,15 @@ int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   ChunkConfig cfg;
-  rc = chunk_tc_config<GATED>(dev, p.T, props, &cfg);
+  rc = chunk_tc_config<GATED, VK>(dev, p.T, props, &cfg);
   if (rc != GDR_OK) return rc;
   CUtensorMap map;
-  rc = encode_pool_map(p, gdr::kTcDK, gdr::kTcVS, false, &map);
+  rc = encode_pool_map(p, gdr::kTcDK, gdr::kTcVS, VK, &map);
   if (rc != GDR_OK) return rc;
   const int n_tiles = p.B * p.H_v * (p.D_v / gdr::kTcVS);
   const int grid = n_tiles < props.sms ? n_tiles : props.sms;
-  gdr::decode_chunk_tc_kernel<GATED><<<grid, cfg.threads, cfg.smem, stream>>>(map, p, n_tiles,
-                                                                            cfg.n_stages);
+  gdr::decode_chunk_tc_kernel<GATED, VK><<<grid, cfg.threads, cfg.smem, stream>>>(
+      map, p, n_tiles, cfg.n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
@@ -421,8 +421,9 @@ const SliceKernel* slice_kernels(int D_k, bool one, bool vk, int* n) {
   return one ? k128_one : k128_many;
 }
 
-// Multi-token calls with D_k = 128 and 128-column slices take the
-// tensor-core chunked kernel. Otherwise the column-slice width is the widest
+// With D_k = 128 and 128-column slices, multi-token calls, and every call on
+// a k-contiguous pool, take the tensor-core kernel. Otherwise the column-slice
+// width is the widest
 // width that divides D_v and still gives every SM GDR_MIN_TILES_PER_SM tiles,
 // else the narrowest one; a width whose stage ring does not fit in shared
 // memory (long T) falls back to the next narrower one.
@@ -434,8 +435,11 @@ int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, bool vk, cudaStrea
   if (rc != GDR_OK) return rc;
   int n = 0;
   const bool one = p.T == 1;
-  if (!one && !vk && D_k == gdr::kTcDK && p.D_v % gdr::kTcVS == 0) {
-    rc = gated ? launch_chunk_tc<true>(p, stream) : launch_chunk_tc<false>(p, stream);
+  if ((!one || vk) && D_k == gdr::kTcDK && p.D_v % gdr::kTcVS == 0) {
+    if (vk)
+      rc = gated ? launch_chunk_tc<true, true>(p, stream) : launch_chunk_tc<false, true>(p, stream);
+    else
+      rc = gated ? launch_chunk_tc<true, false>(p, stream) : launch_chunk_tc<false, false>(p, stream);
     if (rc != GDR_ERR_UNSUPPORTED) return rc;
   }
   const SliceKernel* ks = gated ? slice_kernels<true>(D_k, one, vk, &n)

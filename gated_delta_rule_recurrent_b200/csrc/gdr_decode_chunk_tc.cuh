@@ -1,6 +1,9 @@
-// Multi-token decode kernel (T >= 2) with the two whole-tile contractions on
-// the tcgen05 tensor cores, for 128 x 128 tiles of a [pool, H_v, D_k = 128,
-// D_v] state (D_v a multiple of 128).
+// Decode kernel with the two whole-tile contractions on the tcgen05 tensor
+// cores, for 128 x 128 tiles of a D_k = 128 state (D_v a multiple of 128):
+// multi-token calls on a [pool, H_v, D_k, D_v] pool, and every call on a
+// k-contiguous [pool, H_v, D_v, D_k] pool (VK; there the staged tile holds
+// VS rows j of D_k entries, pass 1 reads it K-major, and pass 2 forms D2^T =
+// [delta parts] [e parts]^T so that TMEM lane j holds row j of the new tile).
 //
 // Arithmetic: the chunked form of the four steps of
 // "lite_boost.ops.recurrent_gated_delta_rule" (MindSpore Lite API page,
@@ -116,6 +119,7 @@ constexpr int kTcDL = 16384;
 constexpr int kTcPart = 24576;  // fp32 [4 warps][8][8] partial sums of A and B
 constexpr int kTcA = 25600;     // fp32 [8][8] A_ts at [t][s], s < t
 constexpr int kTcBm = 25856;    // fp32 [8][8] B_ts at [t][s], s <= t
+constexpr int kTcC = 26112;     // fp32 [DK] c (k-contiguous pools: read across rows)
 constexpr int kTcGroupBytes = 26624;
 
 // Three mbarriers per stage (vectors landed, state landed, stage released)
@@ -371,7 +375,43 @@ __device__ __forceinline__ uint32_t tc_phase(int j, int n_groups, int per_group)
   return static_cast<uint32_t>((j / n_groups) / per_group) & 1u;
 }
 
-template <bool GATED>
+// k-contiguous pool: row j of S_n^T, S_n^T[j, i] = c_i S_0^T[j, i] + D2^T[j, i],
+// over the staged tile [D_k / 64][VS rows j][64] (c from shared memory).
+__device__ __forceinline__ void tc_new_state_row_vk(uint8_t* st, uint32_t d2_lane, const float* c,
+                                                    int j) {
+#pragma unroll
+  for (int k = 0; k < kTcDK / 64; ++k) {
+    uint32_t acc[2][32];
+    tmem_ld32(d2_lane + 64 * k, acc[0]);
+    tmem_ld32(d2_lane + 64 * k + 32, acc[1]);
+    uint4* ptr[8];
+    uint4 s0[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      ptr[q] = reinterpret_cast<uint4*>(st + swz_offset<kTcVS>(j, 64 * k + 8 * q));
+      s0[q] = *ptr[q];
+    }
+    tmem_wait_ld();
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t sw[4] = {s0[q].x, s0[q].y, s0[q].z, s0[q].w};
+      const uint32_t* a = &acc[q >> 2][8 * (q & 3)];
+      const ulonglong2* cq = reinterpret_cast<const ulonglong2*>(c + 64 * k + 8 * q);
+      const ulonglong2 c01 = cq[0], c23 = cq[1];
+      const unsigned long long cc[4] = {c01.x, c01.y, c23.x, c23.y};
+      uint32_t nw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 r = upk(fma2(cc[e], pk(bf16_lo(sw[e]), bf16_hi(sw[e])),
+                                  pk(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]))));
+        nw[e] = pack_bf16x2(r.x, r.y);
+      }
+      *ptr[q] = make_uint4(nw[0], nw[1], nw[2], nw[3]);
+    }
+  }
+}
+
+template <bool GATED, bool VK>
 __global__ void __launch_bounds__(kTcMaxThreads, 1)
     decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                            const int n_tiles, const int n_stages) {
@@ -491,8 +531,12 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
               bulk_load(smem_addr(vb + lay.v + t * VS * 2), vsrc + static_cast<size_t>(t) * p.D_v,
                         VS * 2, vbar);
           }
-          tma_load_3d(smem_addr(smem + stage * kTcStateBytes), &pool_map, 0,
-                      (s * p.H_v + h) * DK, slice * VS / 64, sbar);
+          if constexpr (VK)  // VS rows j of D_k entries
+            tma_load_3d(smem_addr(smem + stage * kTcStateBytes), &pool_map, 0,
+                        (s * p.H_v + h) * p.D_v + slice * VS, 0, sbar);
+          else  // D_k rows i of VS entries
+            tma_load_3d(smem_addr(smem + stage * kTcStateBytes), &pool_map, 0,
+                        (s * p.H_v + h) * DK, slice * VS / 64, sbar);
         }
         mbar_arrive(sbar);
       }
@@ -533,7 +577,9 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     const uint64_t b1_desc = umma_desc(smem_addr(gb + kTcB1), 128, 2048, kUmmaInterleave);
     const uint64_t e_desc = umma_desc(smem_addr(gb + kTcE), 128, 512, kUmmaInterleave);
     const uint64_t dl_desc = umma_desc(smem_addr(gb + kTcDL), 128, 512, kUmmaInterleave);
-    constexpr uint32_t idesc1 = umma_idesc_bf16<kTcVS, kTcN1, true, true>();
+    // pass 1: A = S_0^T (M = j), M-major as [pool, H_v, D_k, D_v] stages it,
+    // K-major as [pool, H_v, D_v, D_k] does; pass 2: both operands K-major
+    constexpr uint32_t idesc1 = umma_idesc_bf16<kTcVS, kTcN1, !VK, true>();
     constexpr uint32_t idesc2 = umma_idesc_bf16<kTcDK, kTcVS, false, false>();
     uint32_t mma_phase = 0;
     int held = -1;  // the stage whose new state is still being stored (elected thread)
@@ -581,6 +627,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
           }
         }
         c_row = tc_finalize_any(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
+        if constexpr (VK) reinterpret_cast<float*>(gb + kTcC)[r] = c_row;
       }
       fence_async_smem();
       if (elected && held >= 0) {  // the previous tile's store has read its stage by now
@@ -596,12 +643,19 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       // ---- 2. pass 1 on the tensor cores; A and B on the CUDA cores
       if (L > 0) {
         if (wq == 0) {  // warp-uniform: one lane issues
-          const uint64_t st_desc = umma_desc(smem_addr(st), DK * 128, 1024, kUmmaSwizzle128);
+          // M-major: LBO = the next 64 columns j, SBO = the next 8 rows i; K-major:
+          // SBO = the next 8 rows j, K steps of 32 bytes inside a 128-byte row
+          // and 64 entries i further on in the next [VS][64] block
+          const uint64_t st_desc =
+              VK ? umma_desc(smem_addr(st), 16, 1024, kUmmaSwizzle128)
+                 : umma_desc(smem_addr(st), DK * 128, 1024, kUmmaSwizzle128);
           if (elect_one()) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < DK / 16; ++ks)
-              umma_bf16(d1, umma_desc_advance(st_desc, ks * 2048),
+              umma_bf16(d1,
+                        umma_desc_advance(st_desc, VK ? (ks >> 2) * (VS * 128) + (ks & 3) * 32
+                                                      : ks * 2048),
                         umma_desc_advance(b1_desc, ks * 256), idesc1, ks > 0);
             umma_commit(mbar);
           }
@@ -633,8 +687,10 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < kTcK2 / 16; ++ks)
-              umma_bf16(d2, umma_desc_advance(e_desc, ks * 256),
-                        umma_desc_advance(dl_desc, ks * 256), idesc2, ks > 0);
+              // [pool, H_v, D_k, D_v]: D2 = E Dl^T (lane = row i); [pool, H_v,
+              // D_v, D_k]: D2 = Dl E^T (lane = row j of the k-contiguous tile)
+              umma_bf16(d2, umma_desc_advance(VK ? dl_desc : e_desc, ks * 256),
+                        umma_desc_advance(VK ? e_desc : dl_desc, ks * 256), idesc2, ks > 0);
             umma_commit(mbar);
           }
           __syncwarp();
@@ -642,7 +698,10 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
         mma_phase ^= 1u;
         tc_fence_after();
-        tc_new_state_row(st, d2 + lane_field, c_row, r);
+        if constexpr (VK)
+          tc_new_state_row_vk(st, d2 + lane_field, reinterpret_cast<const float*>(gb + kTcC), r);
+        else
+          tc_new_state_row(st, d2 + lane_field, c_row, r);
         fence_async_smem();
       }
       tc_fence_before();
@@ -651,7 +710,10 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       // released once the store has read it
       if (elected) {
         if (commit) {
-          tma_store_3d(&pool_map, 0, (s * p.H_v + h) * DK, slice * VS / 64, smem_addr(st));
+          if constexpr (VK)
+            tma_store_3d(&pool_map, 0, (s * p.H_v + h) * p.D_v + slice * VS, 0, smem_addr(st));
+          else
+            tma_store_3d(&pool_map, 0, (s * p.H_v + h) * DK, slice * VS / 64, smem_addr(st));
           bulk_commit_group();
         }
         held = stage;

@@ -57,6 +57,9 @@ def test_every_token_count(T):
     (64, 64, 1, 5, 8),
     (128, 64, 7, 7, 1),
     (64, 512, 4, 4, 2),
+    (128, 128, 2, 4, 1),    # one token on the tensor-core path
+    (128, 256, 2, 4, 8),    # two 128-column slices, all 8 tokens
+    (128, 512, 1, 3, 3),    # four slices, multi-query
 ])
 @pytest.mark.parametrize("gated", [False, True])
 def test_ragged_shapes(D_k, D_v, H_qk, H_v, T, gated):
