@@ -1,9 +1,9 @@
 // Decode kernel with the two whole-tile contractions on the tcgen05 tensor
-// cores, for 128 x 128 tiles of a D_k = 128 state (D_v a multiple of 128):
-// multi-token calls on a [pool, H_v, D_k, D_v] pool, and every call on a
-// k-contiguous [pool, H_v, D_v, D_k] pool (VK; there the staged tile holds
-// VS rows j of D_k entries, pass 1 reads it K-major, and pass 2 forms D2^T =
-// [delta parts] [e parts]^T so that TMEM lane j holds row j of the new tile).
+// cores, for 128 x 128 tiles of a D_k = 128 state (D_v a multiple of 128),
+// any token count, on a [pool, H_v, D_k, D_v] pool or a k-contiguous
+// [pool, H_v, D_v, D_k] pool (VK; there the staged tile holds VS rows j of
+// D_k entries, pass 1 reads it K-major, and pass 2 forms D2^T = [delta parts]
+// [e parts]^T so that TMEM lane j holds row j of the new tile).
 //
 // Arithmetic: the chunked form of the four steps of
 // "lite_boost.ops.recurrent_gated_delta_rule" (MindSpore Lite API page,
