@@ -389,35 +389,35 @@ struct SliceKernel {
 // thread count of a block caps the registers ptxas may give a thread (255 up
 // to 256 threads, 168 up to 384, 128 up to 512, 96 up to 640), and a
 // single-token call keeps no state in registers (about 75 of them), so a
-// full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls that
-// the tensor-core kernel does not take use the CUDA-core chunked kernel.
+// full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls use
+// the CUDA-core chunked kernel. These tables serve the calls the tensor-core
+// kernel does not take (D_k = 64, or D_v not a multiple of 128), and are its
+// fallback.
 template <bool GATED>
 const SliceKernel* slice_kernels(int D_k, bool one, bool vk, int* n) {
   static const SliceKernel k64_one[] = {{512, launch_tma<64, 512, 8, GATED>},
                                         {256, launch_tma<64, 256, 8, GATED>},
                                         {128, launch_tma<64, 128, 8, GATED>},
                                         {64, launch_tma<64, 64, 8, GATED>}};
-  static const SliceKernel k128_one[] = {{256, launch_tma<128, 256, 16, GATED>},
-                                         {128, launch_tma<128, 128, 16, GATED>},
-                                         {64, launch_tma<128, 64, 16, GATED>}};
+  // D_k = 128 with D_v a multiple of 128 goes to the tensor-core kernel, so
+  // only 64-column tiles remain for it here
+  static const SliceKernel k128_one[] = {{64, launch_tma<128, 64, 16, GATED>}};
   static const SliceKernel k64_many[] = {{128, launch_chunk<64, 128, GATED, false>},
                                          {64, launch_chunk<64, 64, GATED, false>}};
-  static const SliceKernel k128_many[] = {{128, launch_chunk<128, 128, GATED, false>},
-                                          {64, launch_chunk<128, 64, GATED, false>}};
+  static const SliceKernel k128_many[] = {{64, launch_chunk<128, 64, GATED, false>}};
   // k-contiguous pools: the chunked kernel for every T (one token is L = 1)
   static const SliceKernel k64_vk[] = {{128, launch_chunk<64, 128, GATED, true>},
                                        {64, launch_chunk<64, 64, GATED, true>}};
-  static const SliceKernel k128_vk[] = {{128, launch_chunk<128, 128, GATED, true>},
-                                        {64, launch_chunk<128, 64, GATED, true>}};
+  static const SliceKernel k128_vk[] = {{64, launch_chunk<128, 64, GATED, true>}};
   if (vk) {
-    *n = 2;
+    *n = D_k == 64 ? 2 : 1;
     return D_k == 64 ? k64_vk : k128_vk;
   }
   if (D_k == 64) {
     *n = one ? 4 : 2;
     return one ? k64_one : k64_many;
   }
-  *n = one ? 3 : 2;
+  *n = 1;
   return one ? k128_one : k128_many;
 }
 
