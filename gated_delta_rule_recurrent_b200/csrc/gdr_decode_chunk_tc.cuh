@@ -109,10 +109,12 @@ __host__ __device__ inline TcLayout tc_layout(int T) {
 //   B1  pass-1 B, N-major: 16 bytes = 8 tokens of one part at row i, at
 //       part * 2048 + (i / 8) * 128 + (i % 8) * 16 (LBO 128 along K = i,
 //       SBO 2048 between the 8-column groups of N);
-//   E   pass-2 A, K-major: 16 bytes = 8 tokens of K group kc at row i, at
+//   E   e parts, K-major: 16 bytes = 8 tokens of K group kc at row i, at
 //       (i / 8) * 512 + kc * 128 + (i % 8) * 16 (LBO 128 between the two K
 //       groups of one MMA, SBO 512 between 8-row groups);
-//   DL  pass-2 B, K-major: the same over columns j.
+//   DL  delta parts, K-major: the same over columns j.
+// Pass 2 takes E as A and DL as B on a [pool, H_v, D_k, D_v] pool, and the
+// other way round on a k-contiguous one.
 constexpr int kTcB1 = 0;
 constexpr int kTcE = 8192;
 constexpr int kTcDL = 16384;
