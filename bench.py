@@ -41,10 +41,16 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 DEFAULT_WORKLOAD = 4
+# What the large-batch kernel's traffic record depends on: the single-token
+# kernel's headers, and in gdr_api.cu its launch configuration (the section
+# between the two markers) and its tile-width table.
 KERNEL_SOURCE_FILES = ("gated_delta_rule_recurrent_b200/csrc/gdr_decode.cuh",
                        "gated_delta_rule_recurrent_b200/csrc/gdr_ptx.cuh",
-                       "gated_delta_rule_recurrent_b200/csrc/gdr_decode_tma.cuh",
-                       "gated_delta_rule_recurrent_b200/csrc/gdr_api.cu")
+                       "gated_delta_rule_recurrent_b200/csrc/gdr_decode_tma.cuh")
+LAUNCH_SOURCE = "gated_delta_rule_recurrent_b200/csrc/gdr_api.cu"
+LAUNCH_SECTION = ("// ---------------------------------------------------------------- TMA path",
+                  "// ---------------------------------------------------------------- chunk path")
+LAUNCH_TABLE = "static const SliceKernel k64_one[]"
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gated_B512_H64_64x512_dram.txt")
 
 
@@ -67,6 +73,12 @@ def kernel_source_hash():
     for rel in KERNEL_SOURCE_FILES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(ROOT, LAUNCH_SOURCE)) as f:
+        api = f.read()
+    a, b = api.index(LAUNCH_SECTION[0]), api.index(LAUNCH_SECTION[1])
+    h.update(api[a:b].encode())
+    t = api.index(LAUNCH_TABLE)
+    h.update(api[t:api.index(";", t)].encode())
     return h.hexdigest()
 
 
