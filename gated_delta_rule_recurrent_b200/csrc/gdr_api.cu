@@ -314,7 +314,7 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
   return GDR_OK;
 }
 
-// ---------------------------------------------------------------- tensor-core chunk path (T >= 2, 128 x 128)
+// ---------------------------------------------------------------- tensor-core path (D_k = 128, 128-column tiles, any T)
 
 // One persistent CTA per SM with kTcGroups consumer groups; each group gets
 // as many stages as shared memory holds (at most 4).
