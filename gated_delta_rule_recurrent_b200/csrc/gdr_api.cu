@@ -318,7 +318,7 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
 
 // One persistent CTA per SM with kTcGroups consumer groups; each group gets
 // as many stages as shared memory holds (at most 4).
-template <bool GATED, bool VK>
+template <bool GATED, bool VK, bool SUMS>
 int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   static ChunkConfig cache[kMaxDevices][gdr::kMaxT + 1];
   static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
@@ -326,7 +326,7 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
     *out = cache[dev][T];
     return GDR_OK;
   }
-  auto kernel = gdr::decode_chunk_tc_kernel<GATED, VK>;
+  auto kernel = gdr::decode_chunk_tc_kernel<GATED, VK, SUMS>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          props.smem_optin);
   if (err == cudaSuccess)
@@ -342,7 +342,7 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
   ChunkConfig c;
   c.n_stages = per * ng;
   c.smem = gdr::tc_smem_bytes(T, c.n_stages, ng);
-  c.threads = gdr::kTcMaxThreads;
+  c.threads = gdr::kTcGroups * (gdr::kTcGroupThreads + (SUMS ? 32 : 0)) + 32;
   int resident = 0;
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, c.threads, c.smem);
   if (err != cudaSuccess)
@@ -354,8 +354,8 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
   return GDR_OK;
 }
 
-template <bool GATED, bool VK>
-int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
+template <bool GATED, bool VK, bool SUMS>
+int launch_chunk_tc_sums(const gdr::DecodeParams& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
@@ -363,19 +363,26 @@ int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   ChunkConfig cfg;
-  rc = chunk_tc_config<GATED, VK>(dev, p.T, props, &cfg);
+  rc = chunk_tc_config<GATED, VK, SUMS>(dev, p.T, props, &cfg);
   if (rc != GDR_OK) return rc;
   CUtensorMap map;
   rc = encode_pool_map(p, gdr::kTcDK, gdr::kTcVS, VK, &map);
   if (rc != GDR_OK) return rc;
   const int n_tiles = p.B * p.H_v * (p.D_v / gdr::kTcVS);
   const int grid = n_tiles < props.sms ? n_tiles : props.sms;
-  gdr::decode_chunk_tc_kernel<GATED, VK><<<grid, cfg.threads, cfg.smem, stream>>>(
+  gdr::decode_chunk_tc_kernel<GATED, VK, SUMS><<<grid, cfg.threads, cfg.smem, stream>>>(
       map, p, n_tiles, cfg.n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
   return GDR_OK;
+}
+
+// Single-token calls take the sums-warp form of the kernel.
+template <bool GATED, bool VK>
+int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
+  return p.T == 1 ? launch_chunk_tc_sums<GATED, VK, true>(p, stream)
+                  : launch_chunk_tc_sums<GATED, VK, false>(p, stream);
 }
 
 using LaunchFn = int (*)(const gdr::DecodeParams&, cudaStream_t);

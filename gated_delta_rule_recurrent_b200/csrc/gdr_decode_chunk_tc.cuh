@@ -81,7 +81,8 @@ constexpr int kTcGroupThreads = 128;  // one thread per TMEM lane
 #define GDR_TC_GROUPS 2
 #endif
 constexpr int kTcGroups = GDR_TC_GROUPS;
-constexpr int kTcMaxThreads = kTcGroups * kTcGroupThreads + 32;
+// groups, one sums warp per group (single-token calls), the producer
+constexpr int kTcMaxThreads = kTcGroups * (kTcGroupThreads + 32) + 32;
 constexpr int kTcN1 = 32;  // pass-1 columns: u_hi, u_lo, w_hi, w_lo, 8 tokens each
 constexpr int kTcK2 = 32;  // pass-2 depth: (e_hi, d_hi), (e_hi, d_lo), (e_lo, d_hi), zeros
 // TMEM columns: D2 of group g at 128 g, D1 of group g at 128 NG + 32 g.
@@ -90,7 +91,7 @@ static_assert(kTcGroups * (kTcVS + kTcN1) <= 512, "TMEM holds 512 columns");
 
 // Per-stage vector block (after the stage's state tile), T padded tokens.
 struct TcLayout {
-  int v, k, q, gk, raw, meta, bytes;
+  int v, k, q, gk, raw, meta, ab, bytes;
 };
 __host__ __device__ inline TcLayout tc_layout(int T) {
   TcLayout s;
@@ -100,7 +101,8 @@ __host__ __device__ inline TcLayout tc_layout(int T) {
   s.gk = s.q + T * kTcDK * 2;      // fp32 [T][DK]  gk rows
   s.raw = s.gk + T * kTcDK * 4;    // u32 [8] g or a words, [8] beta or b words, dt_bias, decay_scale
   s.meta = s.raw + 80;             // int32 [4]     length, slot, committed tokens
-  s.bytes = (s.meta + 16 + 127) & ~127;
+  s.ab = s.meta + 16;              // fp32 [8][8] A_ts, then [8][8] B_ts (from a sums warp)
+  s.bytes = (s.ab + 512 + 127) & ~127;
   return s;
 }
 
@@ -124,12 +126,12 @@ constexpr int kTcBm = 25856;    // fp32 [8][8] B_ts at [t][s], s <= t
 constexpr int kTcC = 26112;     // fp32 [DK] c (k-contiguous pools: read across rows)
 constexpr int kTcGroupBytes = 26624;
 
-// Three mbarriers per stage (vectors landed, state landed, stage released)
-// and one per group (its MMAs done).
+// Four mbarriers per stage (vectors landed, state landed, stage released, A
+// and B summed by a sums warp) and one per group (its MMAs done).
 __host__ __device__ inline int tc_smem_bytes(int T, int n_stages, int n_groups) {
   const int vec = (n_stages * tc_layout(T).bytes + 1023) & ~1023;
   return 1024 /* alignment slack */ + n_stages * kTcStateBytes + vec + n_groups * kTcGroupBytes +
-         (3 * n_stages + n_groups) * 8 + 16;
+         (4 * n_stages + n_groups) * 8 + 16;
 }
 
 // Eight fp32 values as bf16 (hi, lo) parts, packed in pairs: hi = bf16(x),
@@ -155,7 +157,7 @@ __device__ __forceinline__ void split_bf16x8(const float (&x)[8], uint4& hi, uin
 // to slot wq (entry (r, col): B_{t=r, s=col} for col <= r, A_{t=col, s=r} for
 // col > r). The gate value g_t sits in lane t. Returns c_i = P_{n-1}[i] (0
 // when n = 0).
-template <int LC>
+template <int LC, bool PAIRS>
 __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& lay, uint8_t* gb,
                                              float g_lane, float scale, int i, int lane, int wq,
                                              int n) {
@@ -198,6 +200,27 @@ __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& 
   *reinterpret_cast<uint4*>(b1 + 4096) = hi;
   *reinterpret_cast<uint4*>(b1 + 6144) = lo;
 
+  if constexpr (!PAIRS) {  // a sums warp forms A and B: only e_s = P_{s->n-1} k_s here
+    float e[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      e[s] = 0.0f;
+      if (s < LC && s < n) {
+        float z = kf[s];
+#pragma unroll
+        for (int t = s + 1; t < LC; ++t)
+          if (t < n) z *= d[t];
+        e[s] = z;
+      }
+    }
+    split_bf16x8(e, hi, lo);
+    uint8_t* ep = gb + kTcE + (i >> 3) * 512 + (i & 7) * 16;
+    *reinterpret_cast<uint4*>(ep) = hi;
+    *reinterpret_cast<uint4*>(ep + 128) = hi;
+    *reinterpret_cast<uint4*>(ep + 256) = lo;
+    *reinterpret_cast<uint4*>(ep + 384) = make_uint4(0u, 0u, 0u, 0u);
+    return c;
+  }
   // e_s = P_{s->n-1} k_s (0 for s >= n) and the sums A_ts = k_s . P_{s->t} k_t,
   // B_ts = k_s . P_{s->t} q^_t over this row, by running products
   float mp[NM];
@@ -241,18 +264,19 @@ __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& 
   return c;
 }
 
+template <bool PAIRS>
 __device__ __forceinline__ float tc_finalize_any(int L, int n, const uint8_t* vb,
                                                  const TcLayout& lay, uint8_t* gb, float g_lane,
                                                  float scale, int i, int lane, int wq) {
   switch (L) {
-    case 1: return tc_finalize<1>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 2: return tc_finalize<2>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 3: return tc_finalize<3>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 4: return tc_finalize<4>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 5: return tc_finalize<5>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 6: return tc_finalize<6>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 7: return tc_finalize<7>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
-    case 8: return tc_finalize<8>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 1: return tc_finalize<1, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 2: return tc_finalize<2, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 3: return tc_finalize<3, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 4: return tc_finalize<4, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 5: return tc_finalize<5, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 6: return tc_finalize<6, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 7: return tc_finalize<7, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
+    case 8: return tc_finalize<8, PAIRS>(vb, lay, gb, g_lane, scale, i, lane, wq, n);
     default: return 0.0f;
   }
 }
@@ -269,6 +293,80 @@ __device__ __forceinline__ void tc_sum_parts(uint8_t* gb, int L, int r) {
   }
 }
 
+// ---------------------------------------------------------------- the L x L sums
+
+// A_ts = k_s . (P_{s->t} k_t) for s < t and B_ts = k_s . (P_{s->t} q^_t) for
+// s <= t, over the DK rows of a tile with L = LC tokens, by one warp: each
+// lane takes rows lane + 32 m and forms its share by running products, and a
+// warp reduce-scatter leaves each sum in one lane, which writes it to `ab`
+// (A at [t][s], then B at [t][s]). The gate value g_t sits in lane t.
+template <int LC>
+__device__ __forceinline__ void tc_pair_sums(const uint8_t* vb, const TcLayout& lay, float* ab,
+                                             float g_lane, float scale, int lane) {
+  constexpr int DK = kTcDK;
+  constexpr int NM = pow2_at_least(LC * LC);  // padded for the reduce-scatter
+  float g[LC];
+#pragma unroll
+  for (int t = 0; t < LC; ++t) g[t] = __shfl_sync(0xffffffffu, g_lane, t);
+  const uint16_t* sk = reinterpret_cast<const uint16_t*>(vb + lay.k);
+  const uint16_t* sq = reinterpret_cast<const uint16_t*>(vb + lay.q);
+  const float* sgk = reinterpret_cast<const float*>(vb + lay.gk);
+  // mp[s * LC + t] (s < t) holds A_ts, mp[t * LC + s] (s <= t) holds B_ts
+  float mp[NM];
+#pragma unroll
+  for (int j = 0; j < NM; ++j) mp[j] = 0.0f;
+#pragma unroll 1
+  for (int i = lane; i < DK; i += 32) {
+    float d[LC], kf[LC], qf[LC];
+#pragma unroll
+    for (int t = 0; t < LC; ++t) {
+      d[t] = expf(g[t] + sgk[t * DK + i]);
+      kf[t] = bf16_bits_to_f32(sk[t * DK + i]);
+      qf[t] = bf16_bits_to_f32(sq[t * DK + i]) * scale;
+    }
+#pragma unroll
+    for (int s = 0; s < LC; ++s) {
+      float z = kf[s];  // P_{s->t} k_s by running products
+      mp[s * LC + s] = fmaf(z, qf[s], mp[s * LC + s]);
+#pragma unroll
+      for (int t = s + 1; t < LC; ++t) {
+        z *= d[t];
+        mp[s * LC + t] = fmaf(z, kf[t], mp[s * LC + t]);
+        mp[t * LC + s] = fmaf(z, qf[t], mp[t * LC + s]);
+      }
+    }
+  }
+  reduce_scatter<NM>(mp, lane);
+  constexpr int NL = NM >= 32 ? NM / 32 : 1;
+  if (reduce_scatter_writer<NM>(lane)) {
+    const int base = reduce_scatter_base<NM>(lane);
+#pragma unroll
+    for (int j = 0; j < NL; ++j) {
+      const int f = base + j;
+      if (f < LC * LC) {
+        const int r = f / LC, col = f % LC;
+        if (col > r) ab[col * 8 + r] = mp[j];  // A_{t = col, s = r}
+        else ab[64 + r * 8 + col] = mp[j];     // B_{t = r, s = col}
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tc_pair_sums_any(int L, const uint8_t* vb, const TcLayout& lay,
+                                                 float* ab, float g_lane, float scale, int lane) {
+  switch (L) {
+    case 1: tc_pair_sums<1>(vb, lay, ab, g_lane, scale, lane); break;
+    case 2: tc_pair_sums<2>(vb, lay, ab, g_lane, scale, lane); break;
+    case 3: tc_pair_sums<3>(vb, lay, ab, g_lane, scale, lane); break;
+    case 4: tc_pair_sums<4>(vb, lay, ab, g_lane, scale, lane); break;
+    case 5: tc_pair_sums<5>(vb, lay, ab, g_lane, scale, lane); break;
+    case 6: tc_pair_sums<6>(vb, lay, ab, g_lane, scale, lane); break;
+    case 7: tc_pair_sums<7>(vb, lay, ab, g_lane, scale, lane); break;
+    case 8: tc_pair_sums<8>(vb, lay, ab, g_lane, scale, lane); break;
+    default: break;
+  }
+}
+
 // ---------------------------------------------------------------- column-wise: solve
 
 // Column j of a tile with L = LC tokens, from this thread's TMEM lane of D1:
@@ -278,10 +376,9 @@ __device__ __forceinline__ void tc_sum_parts(uint8_t* gb, int L, int r) {
 // lane t.
 template <int LC>
 __device__ __forceinline__ void tc_solve(const uint32_t (&x)[32], const uint8_t* vb,
-                                         const TcLayout& lay, uint8_t* gb, float b_lane, int j,
-                                         uint16_t* out_t0, int D_v) {
-  const float* sa = reinterpret_cast<const float*>(gb + kTcA);
-  const float* sb = reinterpret_cast<const float*>(gb + kTcBm);
+                                         const TcLayout& lay, uint8_t* gb, const float* sa,
+                                         const float* sb, float b_lane, int j, uint16_t* out_t0,
+                                         int D_v) {
   const uint16_t* sv = reinterpret_cast<const uint16_t*>(vb + lay.v);
   float dl[8];
 #pragma unroll
@@ -310,17 +407,18 @@ __device__ __forceinline__ void tc_solve(const uint32_t (&x)[32], const uint8_t*
 }
 
 __device__ __forceinline__ void tc_solve_any(int L, const uint32_t (&x)[32], const uint8_t* vb,
-                                             const TcLayout& lay, uint8_t* gb, float b_lane,
-                                             int j, uint16_t* out_t0, int D_v) {
+                                             const TcLayout& lay, uint8_t* gb, const float* sa,
+                                             const float* sb, float b_lane, int j,
+                                             uint16_t* out_t0, int D_v) {
   switch (L) {
-    case 1: tc_solve<1>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 2: tc_solve<2>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 3: tc_solve<3>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 4: tc_solve<4>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 5: tc_solve<5>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 6: tc_solve<6>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 7: tc_solve<7>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
-    case 8: tc_solve<8>(x, vb, lay, gb, b_lane, j, out_t0, D_v); break;
+    case 1: tc_solve<1>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 2: tc_solve<2>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 3: tc_solve<3>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 4: tc_solve<4>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 5: tc_solve<5>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 6: tc_solve<6>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 7: tc_solve<7>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
+    case 8: tc_solve<8>(x, vb, lay, gb, sa, sb, b_lane, j, out_t0, D_v); break;
     default: break;
   }
 }
@@ -364,8 +462,14 @@ __device__ __forceinline__ void tc_new_state_row(uint8_t* st, uint32_t d2_lane, 
 
 // ---------------------------------------------------------------- kernel
 
-// Block: n_groups = (blockDim.x / 32 - 1) / 4 consumer groups (warps 0 ..
-// 4 n_groups - 1), then the producer warp. Each group owns n_stages / n_groups
+// Block: n_groups consumer groups (warps 0 .. 4 n_groups - 1), then, when
+// SUMS, one sums warp per group, then the producer warp. Sums warp g takes
+// group g's tiles in order, so it follows that group's stages fill by fill
+// and none of its waits can see a phase two fills old either (SUMS serves
+// single-token calls: there the sums are one dot product per tile, and
+// taking them off the groups saves a barrier per tile; with several tokens
+// the sums are the larger part of the row work and are better spread over the
+// groups' four warps, one per scheduler). Each group owns n_stages / n_groups
 // stages (n_stages a multiple of n_groups) and takes them in turn, so a stage
 // passes only between the producer and one group, which has waited for the
 // stage's previous fill before it waits for the next: no wait can see a phase
@@ -413,7 +517,7 @@ __device__ __forceinline__ void tc_new_state_row_vk(uint8_t* st, uint32_t d2_lan
   }
 }
 
-template <bool GATED, bool VK>
+template <bool GATED, bool VK, bool SUMS>
 __global__ void __launch_bounds__(kTcMaxThreads, 1)
     decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                            const int n_tiles, const int n_stages) {
@@ -426,19 +530,21 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
   uint8_t* smem = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
   uint8_t* vec_base = smem + n_stages * kTcStateBytes;
   uint8_t* grp_base = vec_base + ((n_stages * lay.bytes + 1023) & ~1023);
-  const int n_groups = (static_cast<int>(blockDim.x >> 5) - 1) / 4;
+  const int n_groups = (static_cast<int>(blockDim.x >> 5) - 1) / (SUMS ? 5 : 4);
   const int per_group = n_stages / n_groups;
   uint64_t* bars = reinterpret_cast<uint64_t*>(grp_base + n_groups * kTcGroupBytes);
   const uint32_t vec0 = smem_addr(bars);          // k, q, gk, v rows and gate scalars landed
   const uint32_t sta0 = vec0 + 8 * n_stages;      // state tile landed
   const uint32_t empty0 = sta0 + 8 * n_stages;    // the group is done with the stage
-  const uint32_t mma0 = empty0 + 8 * n_stages;    // a group's MMAs are done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * n_stages + n_groups);
+  const uint32_t ab0 = empty0 + 8 * n_stages;     // the stage's A and B are summed (SUMS)
+  const uint32_t mma0 = ab0 + 8 * n_stages;       // a group's MMAs are done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * n_stages + n_groups);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int producer = 4 * n_groups;
+  const int first_sums = 4 * n_groups;  // SUMS: sums warps, one per group
+  const int producer = SUMS ? first_sums + n_groups : first_sums;
   const int n_slices = p.D_v / VS;
   const int n_mine = (n_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
                      static_cast<int>(gridDim.x);
@@ -448,6 +554,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       mbar_init(vec0 + 8 * i, 32);  // one cp.async arrival per producer lane
       mbar_init(sta0 + 8 * i, 1);   // the producer's lane 0 (+ the TMA bytes)
       mbar_init(empty0 + 8 * i, 1); // the group's elected thread
+      mbar_init(ab0 + 8 * i, 1);    // lane 0 of the group's sums warp (SUMS)
     }
     for (int g = 0; g < n_groups; ++g) mbar_init(mma0 + 8 * g, 1);  // one MMA commit
     fence_mbar_init();
@@ -563,7 +670,38 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       }
       cp_async_arrive_noinc(vbar);
     }
-  } else if (warp < producer) {
+  } else if (SUMS && warp >= first_sums) {
+    // ================================================================ the L x L sums
+    for (int j = warp - first_sums; j < n_mine; j += n_groups) {
+      const int tile = blockIdx.x + j * gridDim.x;
+      const int h = (tile / n_slices) % p.H_v;
+      const int b = tile / (n_slices * p.H_v);
+      const int stage = tc_stage(j, n_groups, per_group);
+      const uint8_t* vb = vec_base + stage * lay.bytes;
+      if (!mbar_wait_bounded(vec0 + 8 * stage, tc_phase(j, n_groups, per_group)))
+        flag_error(kErrProducerWait);
+      int L = reinterpret_cast<const int*>(vb + lay.meta)[0];
+      L = L < 0 ? 0 : (L > T ? T : L);
+      if (L > 0) {
+        float gt = 0.0f;
+        if (lane < L) {  // the gate of token `lane` (g only)
+          const uint32_t* rawv = reinterpret_cast<const uint32_t*>(vb + lay.raw);
+          if constexpr (GATED) {
+            const size_t ai = (static_cast<size_t>(b) * T + lane) * p.H_v + h;
+            const float dtb = __uint_as_float(rawv[16]);
+            const float dsc = __uint_as_float(rawv[17]);
+            gt = dsc * softplus_f32(bf16_in_word(rawv[lane], p.gate_a + ai) + dtb);
+          } else {
+            gt = __uint_as_float(rawv[lane]);
+          }
+        }
+        tc_pair_sums_any(L, vb, lay, reinterpret_cast<float*>(const_cast<uint8_t*>(vb) + lay.ab),
+                         gt, p.scale, lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ab0 + 8 * stage);
+    }
+  } else if (warp < first_sums) {
     // ================================================================ consumer groups
     const int group = warp >> 2;
     const int wq = warp & 3;
@@ -628,7 +766,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
             b_lane = bf16_in_word(rawv[8 + lane], p.beta + gi);
           }
         }
-        c_row = tc_finalize_any(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
+        c_row = tc_finalize_any<!SUMS>(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
         if constexpr (VK) reinterpret_cast<float*>(gb + kTcC)[r] = c_row;
       }
       fence_async_smem();
@@ -663,9 +801,15 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
           }
           __syncwarp();
         }
-        tc_sum_parts(gb, L, r);
+        if constexpr (!SUMS) tc_sum_parts(gb, L, r);
       }
-      named_barrier(bar_id, kTcGroupThreads);  // A and B ready
+      if constexpr (SUMS) {
+        // A and B from the sums warp (waited for every tile, so that no later
+        // wait on this stage can see a phase two fills old)
+        if (!mbar_wait_bounded(ab0 + 8 * stage, phase)) flag_error(kErrConsumerWait);
+      } else {
+        named_barrier(bar_id, kTcGroupThreads);  // A and B ready
+      }
 
       // ---- 3. solve: column j = r
       if (L > 0) {
@@ -675,7 +819,10 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         uint32_t x[32];
         tmem_ld32(d1 + lane_field, x);
         tmem_wait_ld();
-        tc_solve_any(L, x, vb, lay, gb, b_lane, r, out_t0, p.D_v);
+        const float* sa = SUMS ? reinterpret_cast<const float*>(vb + lay.ab)
+                               : reinterpret_cast<const float*>(gb + kTcA);
+        const float* sb = SUMS ? sa + 64 : reinterpret_cast<const float*>(gb + kTcBm);
+        tc_solve_any(L, x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
       }
       fence_async_smem();
       tc_fence_before();
