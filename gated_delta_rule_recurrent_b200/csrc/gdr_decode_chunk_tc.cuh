@@ -31,21 +31,24 @@
 // B_ts, the gate, the decays and the unit lower-triangular solve for delta
 // stay on the CUDA cores.
 //
-// CTA: NG consumer groups of 4 warps and one producer warp, one CTA per SM,
-// persistent over tiles blockIdx.x, + gridDim.x, ...; group g takes every
-// NG-th tile. Thread r of a group (warp w = r / 32, so TMEM lanes 32 (w % 4)
-// + lane) is row i = r of the tile in the row-wise steps and column j = r in
-// the column-wise ones:
+// CTA: NG consumer groups of 4 warps and one producer warp (plus, for
+// single-token calls, one sums warp per group), one CTA per SM, persistent
+// over tiles blockIdx.x, + gridDim.x, ...; group g takes every NG-th tile.
+// Thread r of a group (warp w = r / 32, so TMEM lanes 32 (w % 4) + lane) is
+// row i = r of the tile in the row-wise steps and column j = r in the
+// column-wise ones:
 //   1. finalise (row i): decays, u, w, e, c, and its share of A and B (a warp
-//      reduce-scatter into the warp's slot); the pass-1 and pass-2 A operands
-//      go to the group's shared block;
-//   2. one elected thread issues pass 1 (8 MMAs, K = 16 each) and commits it
-//      to the group's mbarrier; threads 0..63 add the four warps' slots of A
-//      and B in a fixed order (deterministic);
+//      reduce-scatter into the warp's slot); the row's pass-1 and pass-2
+//      operands go to the group's shared block;
+//   2. an elected lane issues pass 1 (8 MMAs, K = 16 each) and commits it to
+//      the group's mbarrier; threads 0..63 add the four warps' slots of A and
+//      B in a fixed order (deterministic). For a single token A and B reduce
+//      to B_00 = k . q^, and the group's sums warp forms it instead, so the
+//      group skips the slots and a barrier;
 //   3. solve (column j): reads its TMEM lane of D1 (kv_mem and o parts),
 //      solves for delta, writes o, and writes its delta row of the pass-2 B
 //      operand;
-//   4. the elected thread issues pass 2 (2 MMAs); each thread then reads its
+//   4. the elected lane issues pass 2 (2 MMAs); each thread then reads its
 //      row of D2, adds c_i S_0[i, :] from the staged tile, rounds to bf16 and
 //      writes the row back over S_0 in place; the elected thread stores the
 //      tile to the slot with one TMA store and releases the stage once the
@@ -152,11 +155,11 @@ __device__ __forceinline__ void split_bf16x8(const float (&x)[8], uint4& hi, uin
 
 // ---------------------------------------------------------------- row-wise: finalise
 
-// Row i of a tile with L = LC tokens: writes the pass-1 B operand (u, w) and
-// the pass-2 A operand (e) of the row, and this warp's partial sums of A and B
-// to slot wq (entry (r, col): B_{t=r, s=col} for col <= r, A_{t=col, s=r} for
-// col > r). The gate value g_t sits in lane t. Returns c_i = P_{n-1}[i] (0
-// when n = 0).
+// Row i of a tile with L = LC tokens: writes the row's pass-1 operand (u, w)
+// and pass-2 operand (e), and, when PAIRS, this warp's partial sums of A and
+// B to slot wq (entry (r, col): B_{t=r, s=col} for col <= r, A_{t=col, s=r}
+// for col > r; without PAIRS a sums warp forms them). The gate value g_t sits
+// in lane t. Returns c_i = P_{n-1}[i] (0 when n = 0).
 template <int LC, bool PAIRS>
 __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& lay, uint8_t* gb,
                                              float g_lane, float scale, int i, int lane, int wq,
