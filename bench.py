@@ -6,11 +6,14 @@ scatter) over one batch of seeded synthetic inputs of the large-batch workload
 (B=512 items, 64 heads, T=1, 64x512 bfloat16 state per head, 2 GiB pool).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdr|reference]
+                    [--all-workloads] [--op decode|gate]
 
-Prints one JSON line (rank 0). Multi-GPU: one process per GPU under torchrun;
-each rank decodes its own independent batch and pool (weak scaling, no
-collective on the data path); the timed region is bracketed by barriers and
-the max over ranks is reported.
+Prints one JSON line (rank 0); --all-workloads adds one line for each of the
+single-sequence, grouped-head and speculative workloads after it. Multi-GPU:
+one process per GPU under torchrun; one logical call of N x 512 items is
+split by item over the ranks (each holds its items' pool slots; weak
+scaling, no collective on the data path); the timed region is bracketed by
+barriers and the max over ranks is reported.
 
 ``--impl reference`` times the CPU oracle (fp64 NumPy) on this machine's host
 cores on a bounded sample of the same workload; it is a deliberately slow
@@ -117,7 +120,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int, period_ms: int = 50):
+    def __init__(self, device_index: int, period_ms: int = 10):
         self.samples = []  # (host time, sm_mhz, max_mhz, power, reasons set)
         self.proc = None
         try:
@@ -291,41 +294,60 @@ def measure_e2e(args, w, x, xd, out, dev, step, barrier, max_over_ranks, world, 
 
 # --------------------------------------------------------------------------- CUDA arm
 
-def run_gdr(args):
-    import torch.distributed as dist
+def _place(x, dev, layout):
+    """Device copies of one call's inputs (the pool in the requested layout)."""
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    if layout == "vk":  # the same state, stored [pool, H_v, D_v, D_k]
+        xd["state_pool"] = xd["state_pool"].transpose(2, 3).contiguous()
+    return xd
 
-    world, rank, local = distributed.rank_env()
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
 
-        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+def _timed_region(step, K, stream, dev, barrier, max_over_ranks):
+    """K steps back to back between two events on the launching stream,
+    bracketed by a barrier and a device synchronisation on both sides; the
+    max over ranks of the region, and the host times of its ends."""
+    r0 = torch.cuda.Event(enable_timing=True)
+    r1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    host_t0 = time.time()
+    r0.record(stream)
+    for i in range(K):
+        step(i)
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    host_t1 = time.time()
+    barrier()
+    return max_over_ranks(r0.elapsed_time(r1)), host_t0, host_t1
 
+
+def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
+    """One JSON line for one decode workload on this rank's GPU."""
     import gated_delta_rule_recurrent_b200 as gdr
-    from gated_delta_rule_recurrent_b200 import binding
 
-    binding.lib()  # fail loudly now if the library is missing
-    w = workloads.workload(args.workload)
-    if args.batch is not None:
+    world, rank, dev, barrier, max_over_ranks, sampler = ctx
+    w = workloads.workload(wkey)
+    if args.batch is not None and wkey == args.workload:
         w = w.replace(name=f"{w.name}_B{args.batch}", B=args.batch, pool=args.batch)
     gated = w.gated
-    # Each rank decodes its own batch: independent sequences and pool slots.
+    # One logical call of N x B items over N x pool slots, split by item
+    # (distributed.shard_call's contiguous item split): rank r holds items
+    # [r B, (r + 1) B) and the slots they name. Its share is drawn from its own
+    # seed, so no rank builds the others' inputs.
     x = workloads.make_inputs(w, seed=distributed.rank_seed(w.seed, rank))
-    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    if args.layout == "vk":  # the same state, stored [pool, H_v, D_v, D_k]
-        xd["state_pool"] = xd["state_pool"].transpose(2, 3).contiguous()
-    out = torch.empty(w.B, w.H_v, w.T, w.D_v, dtype=torch.bfloat16, device=dev)
     lengths = x["actual_seq_lengths"].tolist()
     n_tokens = int(sum(min(max(L, 0), w.T) for L in lengths))
     step_bytes = metrics.algorithmic_bytes(w.B, w.H_qk, w.H_v, w.T, w.D_k, w.D_v, lengths,
                                            gated)
+    # Every step must read its inputs from HBM: a workload smaller than a few
+    # L2s rotates over copies of its inputs and pool that together exceed it.
+    n_copies = max(1, min(64, math.ceil(3 * L2_BYTES / step_bytes)))
+    copies = [_place(x, dev, args.layout) for _ in range(n_copies)]
+    outs = [torch.empty(w.B, w.H_v, w.T, w.D_v, dtype=torch.bfloat16, device=dev)
+            for _ in range(n_copies)]
     stream = torch.cuda.current_stream(dev)
 
-    def step(o=out, inputs=None):
-        z = xd if inputs is None else {**xd, **inputs}
+    def call(z, o):
         if gated:
             gdr.decode_gated(z["query"], z["key"], z["value"], z["a"], z["b"],
                              z["dt_bias"], z["decay_scale"], z["state_pool"],
@@ -338,70 +360,61 @@ def run_gdr(args):
                        z["num_accepted_tokens"], z["scale_value"], out=o,
                        state_layout=args.layout)
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
-
-    def max_over_ranks(v):
-        return distributed.max_over_ranks(v, dev)
-
-    sampler = ClockSampler(local)
-    sampler.wait_first()
+    def step(i):
+        call(copies[i % n_copies], outs[i % n_copies])
 
     # ---- kernel-resident timing: inputs already in HBM
-    for _ in range(args.warmup):
-        step()
+    for i in range(max(args.warmup, n_copies)):
+        step(i)
     torch.cuda.synchronize(dev)
+    kernel = gdr.last_launch()
+    K = args.steps
     # Events only at the two ends of the region: the steps run back to back
     # (the host enqueues a call in ~25 us, ahead of the device), one decode
     # launch per step, so the average launch duration is the region over the
     # launches. (An event pair around every launch leaves the device idle for
     # a few microseconds between launches, which a short step would count.)
-    K = args.steps
-    region0 = torch.cuda.Event(enable_timing=True)
-    region1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    host_t0 = time.time()
-    region0.record(stream)
-    for i in range(K):
-        step()
-    region1.record(stream)
-    torch.cuda.synchronize(dev)
-    host_t1 = time.time()
-    barrier()
+    region_ms, host_t0, host_t1 = _timed_region(step, K, stream, dev, barrier, max_over_ranks)
+    clocks = sampler.summary(host_t0, host_t1)
+    # the same region again, back to back: its spread shows the run's noise
+    repeats = [_timed_region(step, K, stream, dev, barrier, max_over_ranks)[0] / K
+               for _ in range(args.repeats)]
     launches = K  # one kernel per step (the decode kernel)
-    region_ms = max_over_ranks(region0.elapsed_time(region1))
     total_tokens = distributed.sum_over_ranks(n_tokens * K, dev)
     kernel_ms = region_ms / launches
-    clocks = sampler.summary(host_t0, host_t1)
 
     # ---- end to end through the public API: pinned host inputs copied in and
     # the output copied back every step, inside the timed region. The state
     # pool stays resident on the device, as it does in serving.
     e2e = None
-    if not args.no_e2e:
-        e2e = measure_e2e(args, w, x, xd, out, dev, step, barrier, max_over_ranks, world,
+    if with_e2e:
+        xd = copies[0]
+        out = outs[0]
+
+        def e2e_step(o=out, inputs=None):
+            call({**xd, **inputs} if inputs is not None else xd, o)
+
+        e2e = measure_e2e(args, w, x, xd, out, dev, e2e_step, barrier, max_over_ranks, world,
                           n_tokens)
-    sampler.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, toks, items, secs = oracle_tokens_per_s(x, gated, items_per_call=8,
-                                                     budget_s=args.cpu_seconds)
+                                                     budget_s=cpu_seconds)
         cpu = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": f"{items} of {w.B} batch items ({toks} tokens) of the same "
                          f"workload, fp64 NumPy, 1 thread, {secs:.1f} s of oracle time"}
-
-    if world > 1:
-        dist.destroy_process_group()
-    if rank != 0:
-        return
+    del copies, outs
 
     peak, peak_kind = measured_hbm_peak()
     achieved = step_bytes / (kernel_ms / 1e3) / 1e9
     value = total_tokens / (region_ms / 1e3)
-    line = {
+    l2 = (f"inputs larger than L2: {step_bytes / 1e9:.2f} GB per step vs "
+          f"{L2_BYTES / 2**20:.0f} MiB L2, no flush" if n_copies == 1 else
+          f"{step_bytes / 1e6:.1f} MB per step: steps rotate over {n_copies} copies of the "
+          f"inputs and pool ({n_copies * step_bytes / 1e6:.0f} MB, over 3x the "
+          f"{L2_BYTES / 2**20:.0f} MiB L2), no flush")
+    return {
         "metric": METRIC,
         "value": value,
         "unit": "tokens/s",
@@ -417,28 +430,75 @@ def run_gdr(args):
         "config": {
             "workload": w.name, "B": w.B, "H_qk": w.H_qk, "H_v": w.H_v, "T": w.T,
             "D_k": w.D_k, "D_v": w.D_v, "pool": w.pool,
+            "tokens_per_step": n_tokens,
             "gate": "fused" if gated else "none",
             "storage": "bf16 state/q/k/v/out, fp32 g/gk",
             "state_layout": "[pool, H_v, D_k, D_v]" if args.layout == "kv"
                             else "[pool, H_v, D_v, D_k]",
-            "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB per step vs "
-                  f"{L2_BYTES / 2**20:.0f} MiB L2, no flush",
-            "parallelism": f"{world} independent rank(s), no collective",
+            "l2": l2,
+            "parallelism": f"one call of {world} x {w.B} items split by item over {world} "
+                           f"rank(s), no collective",
         },
         "achieved_hbm_gbs": achieved,
         "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+        "repeat_ms_per_step": {
+            "n": len(repeats), "median": float(np.median(repeats)) if repeats else None,
+            "min": min(repeats) if repeats else None, "max": max(repeats) if repeats else None,
+            "note": f"{len(repeats)} more regions of {K} steps right after the timed one"},
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth",
             "kernel": decode_kernel_name(w, args.layout), "kernel_ms": kernel_ms,
-            "bytes_per_launch": step_bytes, "traffic": recorded_traffic(w.name, args.layout),
+            "kernel_form": kernel,
+            "bytes_per_launch": step_bytes,
+            "traffic": recorded_traffic(w.name, args.layout) if n_copies == 1 else None,
         },
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
-    print(json.dumps(line), flush=True)
+
+
+def run_gdr(args):
+    import torch.distributed as dist
+
+    world, rank, local = distributed.rank_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    from gated_delta_rule_recurrent_b200 import binding
+
+    binding.lib()  # fail loudly now if the library is missing
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v):
+        return distributed.max_over_ranks(v, dev)
+
+    sampler = ClockSampler(local, period_ms=10)
+    sampler.wait_first()
+    ctx = (world, rank, dev, barrier, max_over_ranks, sampler)
+    lines = [bench_decode_workload(args, args.workload, ctx, not args.no_e2e, args.cpu_seconds)]
+    if args.all_workloads:
+        for wk in (1, 2, 3):
+            if wk != args.workload:
+                lines.append(bench_decode_workload(args, wk, ctx, False,
+                                                   min(args.cpu_seconds, 5.0)))
+    sampler.stop()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        for line in lines:
+            print(json.dumps(line), flush=True)
 
 
 # --------------------------------------------------------------------------- oracle arm
@@ -593,6 +653,12 @@ def main():
     ap.add_argument("--gate-shape", default="32768x8x64",
                     help="shape of a and b for --op gate, heads last")
     ap.add_argument("--gate-dtype", choices=("f32", "f16", "bf16"), default="bf16")
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="after the default line, one line for each of workloads 1-3 (the "
+                         "single-sequence, grouped-head and speculative decode workloads)")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="extra timed regions after the main one, reported as "
+                         "repeat_ms_per_step (the main region alone gives ms_per_step)")
     ap.add_argument("--layout", choices=("kv", "vk"), default="kv",
                     help="state pool layout: kv = [pool, H_v, D_k, D_v] (the op page's), "
                          "vk = [pool, H_v, D_v, D_k]")

@@ -15,9 +15,10 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["decode", "decode_gated", "linear_attention_gate", "device_error", "GdrError", "lib",
-           "library_path",
-           "STATUS_NAMES", "Dims"]
+__all__ = ["decode", "decode_gated", "prefill", "prefill_gated", "linear_attention_gate",
+           "device_error", "GdrError", "lib",
+           "library_path", "last_launch", "kernel_forms", "KERNEL_NAMES",
+           "STATUS_NAMES", "Dims", "LaunchInfo"]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 
@@ -38,6 +39,23 @@ class Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32)
                 for n in ("B", "T", "H_qk", "H_v", "D_k", "D_v", "pool_size", "layout")]
 
+
+class LaunchInfo(ctypes.Structure):
+    """gdr_launch_info: one kernel launch (or one kernel form of the dispatcher)."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "D_k", "tile_cols", "gated", "layout",
+                                              "grid", "threads", "smem_bytes", "stages")]
+
+    def as_dict(self) -> dict:
+        d = {n: int(getattr(self, n)) for n, _ in self._fields_}
+        d["kernel"] = KERNEL_NAMES.get(d["kernel"], d["kernel"])
+        d["layout"] = "vk" if d["layout"] == 1 else "kv"
+        d["gated"] = bool(d["gated"])
+        return d
+
+
+# gdr_kernel values of include/gdr.h
+KERNEL_NAMES = {0: "none", 1: "single_token", 2: "chunked", 3: "tensor_core",
+                4: "tensor_core_one", 5: "gate", 6: "prefill"}
 
 _P = ctypes.c_void_p
 _DECODE_ARGTYPES = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -66,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.gdr_decode.restype = ctypes.c_int
         L.gdr_gate_fused.argtypes = _GATED_ARGTYPES
         L.gdr_gate_fused.restype = ctypes.c_int
+        L.gdr_prefill.argtypes = _DECODE_ARGTYPES
+        L.gdr_prefill.restype = ctypes.c_int
+        L.gdr_prefill_gated.argtypes = _GATED_ARGTYPES
+        L.gdr_prefill_gated.restype = ctypes.c_int
         L.gdr_status_string.argtypes = [ctypes.c_int]
         L.gdr_status_string.restype = ctypes.c_char_p
         L.gdr_last_error.argtypes = []
@@ -78,6 +100,12 @@ def lib() -> ctypes.CDLL:
         L.gdr_linear_attention_gate.argtypes = [P, P, P, P, P, P, ctypes.c_int64, ctypes.c_int32,
                                                 ctypes.c_int, P]
         L.gdr_linear_attention_gate.restype = ctypes.c_int
+        L.gdr_last_launch.argtypes = [ctypes.POINTER(LaunchInfo)]
+        L.gdr_last_launch.restype = ctypes.c_int
+        L.gdr_kernel_form_count.argtypes = []
+        L.gdr_kernel_form_count.restype = ctypes.c_int
+        L.gdr_kernel_form.argtypes = [ctypes.c_int, ctypes.POINTER(LaunchInfo)]
+        L.gdr_kernel_form.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -95,6 +123,28 @@ def device_error(reset: bool = True, device=None) -> int:
         rc = lib().gdr_device_error(ctypes.byref(flags), int(bool(reset)))
     _check(rc)
     return int(flags.value)
+
+
+def last_launch() -> dict:
+    """The calling thread's most recent kernel launch through the library
+    (``gdr_last_launch``): kernel family, D_k, tile columns, gate, layout and
+    the launch shape. ``kernel`` is "none" after a call that queued nothing."""
+    info = LaunchInfo()
+    _check(lib().gdr_last_launch(ctypes.byref(info)))
+    return info.as_dict()
+
+
+def kernel_forms() -> list:
+    """Every decode kernel form the dispatcher can choose (``gdr_kernel_form``),
+    as dicts with kernel, D_k, tile_cols, gated and layout. Needs no GPU."""
+    L = lib()
+    forms = []
+    for i in range(L.gdr_kernel_form_count()):
+        info = LaunchInfo()
+        _check(L.gdr_kernel_form(i, ctypes.byref(info)))
+        d = info.as_dict()
+        forms.append({k: d[k] for k in ("kernel", "D_k", "tile_cols", "gated", "layout")})
+    return forms
 
 
 def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape, device) -> None:
@@ -217,6 +267,54 @@ def decode_gated(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, a:
                                   _ptr(ssm_state_indices), _ptr(gk),
                                   _ptr(num_accepted_tokens), float(scale_value), _ptr(out),
                                   stream)
+    _check(rc)
+    return out, state_pool
+
+
+def prefill(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, beta: torch.Tensor,
+            state_pool: torch.Tensor, actual_seq_lengths: torch.Tensor,
+            ssm_state_indices: torch.Tensor, g: torch.Tensor, gk: torch.Tensor,
+            num_accepted_tokens: Optional[torch.Tensor] = None, scale_value: float = 1.0, *,
+            out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The recurrence over a long prompt through ``gdr_prefill``: the arguments
+    and results of ``decode`` for any token count T (D_k = 128, D_v a multiple
+    of 128, the [pool, H_v, D_k, D_v] pool)."""
+    device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
+                                        ssm_state_indices, gk, num_accepted_tokens, out, "kv")
+    B, H_v, T = dims.B, dims.H_v, dims.T
+    _need(beta, "beta", torch.bfloat16, (B, H_v, T), device)
+    _need(g, "g", torch.float32, (B, H_v, T), device)
+    with torch.cuda.device(device):
+        rc = lib().gdr_prefill(ctypes.byref(dims), _ptr(query), _ptr(key), _ptr(value),
+                               _ptr(beta), _ptr(state_pool), _ptr(actual_seq_lengths),
+                               _ptr(ssm_state_indices), _ptr(g), _ptr(gk),
+                               _ptr(num_accepted_tokens), float(scale_value), _ptr(out), stream)
+    _check(rc)
+    return out, state_pool
+
+
+def prefill_gated(query: torch.Tensor, key: torch.Tensor, value: torch.Tensor, a: torch.Tensor,
+                  b: torch.Tensor, dt_bias: torch.Tensor, decay_scale: torch.Tensor,
+                  state_pool: torch.Tensor, actual_seq_lengths: torch.Tensor,
+                  ssm_state_indices: torch.Tensor, gk: torch.Tensor,
+                  num_accepted_tokens: Optional[torch.Tensor] = None, scale_value: float = 1.0,
+                  *, out: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """``prefill`` with the LinearAttentionGate fused, through ``gdr_prefill_gated``
+    (the gate arguments of ``decode_gated``)."""
+    device, dims, out, stream = _common(query, key, value, state_pool, actual_seq_lengths,
+                                        ssm_state_indices, gk, num_accepted_tokens, out, "kv")
+    B, H_v, T = dims.B, dims.H_v, dims.T
+    _need(a, "a", torch.bfloat16, (B, T, H_v), device)
+    _need(b, "b", torch.bfloat16, (B, T, H_v), device)
+    _need(dt_bias, "dt_bias", torch.float32, (H_v,), device)
+    _need(decay_scale, "decay_scale", torch.float32, (H_v,), device)
+    with torch.cuda.device(device):
+        rc = lib().gdr_prefill_gated(ctypes.byref(dims), _ptr(query), _ptr(key), _ptr(value),
+                                     _ptr(a), _ptr(b), _ptr(dt_bias), _ptr(decay_scale),
+                                     _ptr(state_pool), _ptr(actual_seq_lengths),
+                                     _ptr(ssm_state_indices), _ptr(gk),
+                                     _ptr(num_accepted_tokens), float(scale_value), _ptr(out),
+                                     stream)
     _check(rc)
     return out, state_pool
 

@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "gdr.h"
 #include "gdr_decode.cuh"
@@ -21,10 +22,18 @@
 #include "gdr_decode_chunk_tc.cuh"
 #include "gdr_decode_tma.cuh"
 #include "gdr_gate.cuh"
+#include "gdr_prefill_tc.cuh"
 
 namespace {
 
 thread_local std::string g_last_error;
+thread_local gdr_launch_info g_last_launch{};
+
+void record_launch(int kernel, int D_k, int tile_cols, bool gated, bool vk, int grid,
+                   int threads, int smem, int stages) {
+  g_last_launch = gdr_launch_info{kernel, D_k, tile_cols, gated ? 1 : 0,
+                                  vk ? GDR_LAYOUT_VK : GDR_LAYOUT_KV, grid, threads, smem, stages};
+}
 
 int fail(int status, const std::string& what) {
   g_last_error = what;
@@ -232,6 +241,8 @@ int launch_tma(const gdr::DecodeParams& p, cudaStream_t stream) {
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  record_launch(GDR_KERNEL_SINGLE_TOKEN, DK, VS, GATED, false, grid, Shape::kThreads, smem,
+                n_stages);
   return GDR_OK;
 }
 
@@ -268,7 +279,7 @@ int chunk_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
     return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
   constexpr int kMaxStagesChunk = GDR_CHUNK_MAX_STAGES;
   const int stage_bytes = gdr::chunk_stage_bytes<DK, VS>(T);
-  int n = (props.smem_optin - 1024 - gdr::kChunkBarriers * 8 * kMaxStagesChunk) / stage_bytes;
+  int n = (props.smem_optin - 1024 - gdr::kChunkBarriers * 8 * kMaxStagesChunk - 16) / stage_bytes;
   n = n > kMaxStagesChunk ? kMaxStagesChunk : n;
   if (n < 2) return fail(GDR_ERR_UNSUPPORTED, "tile does not fit in shared memory");
   constexpr int cwt = gdr::ChunkShape<DK, VS, VK>::kWarpsPerTile;
@@ -311,6 +322,8 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  record_launch(GDR_KERNEL_CHUNKED, DK, VS, GATED, VK, grid, cfg.threads, cfg.smem,
+                cfg.n_stages);
   return GDR_OK;
 }
 
@@ -375,6 +388,8 @@ int launch_chunk_tc_sums(const gdr::DecodeParams& p, cudaStream_t stream) {
   err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  record_launch(SUMS ? GDR_KERNEL_TENSOR_CORE_ONE : GDR_KERNEL_TENSOR_CORE, gdr::kTcDK,
+                gdr::kTcVS, GATED, VK, grid, cfg.threads, cfg.smem, cfg.n_stages);
   return GDR_OK;
 }
 
@@ -469,6 +484,34 @@ int dispatch(const gdr::DecodeParams& p, int D_k, bool gated, bool vk, cudaStrea
   return rc;
 }
 
+// Every kernel form the entry points can launch: the prefill kernel, then,
+// per gate variant, the decode dispatcher's: the tensor-core kernel's four
+// (layout x token form), then the entries of the tile-width tables.
+std::vector<gdr_launch_info> kernel_forms() {
+  std::vector<gdr_launch_info> forms;
+  for (int gated = 0; gated < 2; ++gated)  // gdr_prefill / gdr_prefill_gated
+    forms.push_back(gdr_launch_info{GDR_KERNEL_PREFILL, gdr::kTcDK, gdr::kTcVS, gated,
+                                    GDR_LAYOUT_KV, 0, 0, 0, 0});
+  for (int gated = 0; gated < 2; ++gated) {
+    for (int vk = 0; vk < 2; ++vk)
+      for (int kernel : {GDR_KERNEL_TENSOR_CORE_ONE, GDR_KERNEL_TENSOR_CORE})
+        forms.push_back(gdr_launch_info{kernel, gdr::kTcDK, gdr::kTcVS, gated, vk, 0, 0, 0, 0});
+    for (int D_k : {64, 128})
+      for (int vk = 0; vk < 2; ++vk)
+        for (int one = 1; one >= 0; --one) {
+          if (vk && one) continue;  // k-contiguous pools: one table for every T
+          int n = 0;
+          const SliceKernel* ks = gated ? slice_kernels<true>(D_k, one, vk, &n)
+                                        : slice_kernels<false>(D_k, one, vk, &n);
+          for (int i = 0; i < n; ++i)
+            forms.push_back(gdr_launch_info{
+                one && !vk ? GDR_KERNEL_SINGLE_TOKEN : GDR_KERNEL_CHUNKED, D_k, ks[i].vs, gated,
+                vk, 0, 0, 0, 0});
+        }
+  }
+  return forms;
+}
+
 gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gdr_bf16* key,
                               const gdr_bf16* value, gdr_bf16* state_pool,
                               const int32_t* asl, const int32_t* idx, const int32_t* nat,
@@ -492,6 +535,72 @@ gdr::DecodeParams base_params(const gdr_dims* d, const gdr_bf16* query, const gd
   p.pool_size = d->pool_size;
   p.group = d->H_v / d->H_qk;
   return p;
+}
+
+// ---------------------------------------------------------------- prefill (long T)
+
+int check_prefill_dims(const gdr_dims* d) {
+  if (d == nullptr) return fail(GDR_ERR_NULL, "dims is NULL");
+  if (d->B < 0) return fail(GDR_ERR_DIMS, "B must be >= 0");
+  if (d->T < 1) return fail(GDR_ERR_DIMS, "T must be >= 1");
+  if (d->H_qk < 1 || d->H_v < 1) return fail(GDR_ERR_DIMS, "H_qk and H_v must be >= 1");
+  if (d->H_v % d->H_qk != 0) return fail(GDR_ERR_DIMS, "H_v must be a multiple of H_qk");
+  if (d->D_k < 1 || d->D_v < 1) return fail(GDR_ERR_DIMS, "D_k and D_v must be >= 1");
+  if (d->pool_size < 1) return fail(GDR_ERR_DIMS, "pool_size must be >= 1");
+  if (d->layout != GDR_LAYOUT_KV && d->layout != GDR_LAYOUT_VK)
+    return fail(GDR_ERR_DIMS, "layout must be GDR_LAYOUT_KV or GDR_LAYOUT_VK");
+  if (d->D_k != gdr::kTcDK || d->D_v % gdr::kTcVS != 0 || d->layout != GDR_LAYOUT_KV)
+    return fail(GDR_ERR_UNSUPPORTED,
+                "prefill takes D_k = 128, D_v a multiple of 128 and the [pool, H_v, D_k, D_v] "
+                "layout");
+  const long long tiles = static_cast<long long>(d->B) * d->H_v * (d->D_v / gdr::kTcVS);
+  if (tiles > 0x7fffffffLL) return fail(GDR_ERR_DIMS, "B * H_v * D_v / 128 exceeds 2^31 - 1");
+  if (static_cast<long long>(d->pool_size) * d->H_v * d->D_k > 0x7fffffffLL)
+    return fail(GDR_ERR_UNSUPPORTED, "pool_size * H_v * D_k exceeds 2^31 - 1");
+  // element offsets are 64-bit; keep every tensor's element count below 2^62
+  const long long per_item = static_cast<long long>(d->T) *
+                             (d->H_v > d->H_qk ? d->H_v : d->H_qk) *
+                             (d->D_v > d->D_k ? d->D_v : d->D_k);
+  if (per_item > (1LL << 62) / (d->B > 0 ? d->B : 1))
+    return fail(GDR_ERR_DIMS, "B * H * T * D exceeds 2^62");
+  return GDR_OK;
+}
+
+template <bool GATED>
+int launch_prefill(const gdr::DecodeParams& p, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(GDR_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
+  DeviceProps props;
+  int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  const int smem = gdr::pf_smem_bytes();
+  if (smem > props.smem_optin) return fail(GDR_ERR_UNSUPPORTED, "prefill tile does not fit in shared memory");
+  static std::atomic<bool> ready[kMaxDevices];
+  auto kernel = gdr::prefill_tc_kernel<GATED>;
+  if (!ready[dev].load(std::memory_order_acquire)) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (err != cudaSuccess)
+      return fail(GDR_ERR_CUDA, std::string("kernel attributes: ") + cudaGetErrorString(err));
+    ready[dev].store(true, std::memory_order_release);
+  }
+  CUtensorMap map;
+  rc = encode_pool_map(p, gdr::kTcDK, gdr::kTcVS, false, &map);
+  if (rc != GDR_OK) return rc;
+  // One tile per SM while there are fewer tiles than SMs (each tile is a long
+  // sequential chain); past that, a CTA's two groups share an SM.
+  const int n_tiles = p.B * p.H_v * (p.D_v / gdr::kTcVS);
+  const int grid = n_tiles < props.sms ? n_tiles : props.sms;
+  kernel<<<grid, gdr::kPfThreads, smem, stream>>>(map, p, n_tiles);
+  err = cudaGetLastError();
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  record_launch(GDR_KERNEL_PREFILL, gdr::kTcDK, gdr::kTcVS, GATED, false, grid, gdr::kPfThreads,
+                smem, gdr::kPfStages);
+  return GDR_OK;
 }
 
 // ---------------------------------------------------------------- standalone gate
@@ -527,6 +636,8 @@ int launch_gate(const void* a, const void* b, const float* dt_bias, const float*
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  record_launch(GDR_KERNEL_GATE, 0, 0, true, false,
+                n_vec > 0 ? blocks_for(n_vec) : blocks_for(n - i_begin), kThreads, 0, 0);
   return GDR_OK;
 }
 
@@ -559,6 +670,7 @@ GDR_API int gdr_decode(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf
                        const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
                        const float* g, const float* gk, const int32_t* num_accepted_tokens,
                        float scale_value, gdr_bf16* out, gdr_stream_t stream) {
+  g_last_launch = gdr_launch_info{};
   int rc = check_dims(dims);
   if (rc != GDR_OK) return rc;
   if (dims->B == 0) return GDR_OK;
@@ -581,6 +693,7 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
                            const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
                            const float* gk, const int32_t* num_accepted_tokens,
                            float scale_value, gdr_bf16* out, gdr_stream_t stream) {
+  g_last_launch = gdr_launch_info{};
   int rc = check_dims(dims);
   if (rc != GDR_OK) return rc;
   if (dims->B == 0) return GDR_OK;
@@ -600,9 +713,57 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
+GDR_API int gdr_prefill(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
+                        const gdr_bf16* value, const gdr_bf16* beta, gdr_bf16* state_pool,
+                        const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
+                        const float* g, const float* gk, const int32_t* num_accepted_tokens,
+                        float scale_value, gdr_bf16* out, gdr_stream_t stream) {
+  g_last_launch = gdr_launch_info{};
+  int rc = check_prefill_dims(dims);
+  if (rc != GDR_OK) return rc;
+  if (dims->B == 0) return GDR_OK;
+  rc = check_common_pointers(query, key, value, state_pool, actual_seq_lengths,
+                             ssm_state_indices, gk, out);
+  if (rc != GDR_OK) return rc;
+  if (!beta || !g) return fail(GDR_ERR_NULL, "beta and g must not be NULL");
+  gdr::DecodeParams p = base_params(dims, query, key, value, state_pool, actual_seq_lengths,
+                                    ssm_state_indices, num_accepted_tokens, gk, scale_value,
+                                    out);
+  p.beta = beta;
+  p.g = g;
+  return launch_prefill<false>(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+GDR_API int gdr_prefill_gated(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
+                              const gdr_bf16* value, const gdr_bf16* a, const gdr_bf16* b,
+                              const float* dt_bias, const float* decay_scale,
+                              gdr_bf16* state_pool, const int32_t* actual_seq_lengths,
+                              const int32_t* ssm_state_indices, const float* gk,
+                              const int32_t* num_accepted_tokens, float scale_value,
+                              gdr_bf16* out, gdr_stream_t stream) {
+  g_last_launch = gdr_launch_info{};
+  int rc = check_prefill_dims(dims);
+  if (rc != GDR_OK) return rc;
+  if (dims->B == 0) return GDR_OK;
+  rc = check_common_pointers(query, key, value, state_pool, actual_seq_lengths,
+                             ssm_state_indices, gk, out);
+  if (rc != GDR_OK) return rc;
+  if (!a || !b || !dt_bias || !decay_scale)
+    return fail(GDR_ERR_NULL, "a, b, dt_bias and decay_scale must not be NULL");
+  gdr::DecodeParams p = base_params(dims, query, key, value, state_pool, actual_seq_lengths,
+                                    ssm_state_indices, num_accepted_tokens, gk, scale_value,
+                                    out);
+  p.gate_a = a;
+  p.gate_b = b;
+  p.dt_bias = dt_bias;
+  p.decay_scale = decay_scale;
+  return launch_prefill<true>(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
 GDR_API int gdr_linear_attention_gate(const void* a, const void* b, const float* dt_bias,
                                       const float* decay_scale, void* decay, void* beta,
                                       int64_t rows, int32_t H, int dtype, gdr_stream_t stream) {
+  g_last_launch = gdr_launch_info{};
   if (!a || !dt_bias || !decay_scale || !decay)
     return fail(GDR_ERR_NULL, "a, dt_bias, decay_scale and decay must not be NULL");
   if (beta != nullptr && b == nullptr)
@@ -653,6 +814,39 @@ GDR_API int gdr_device_error(uint32_t* flags, int reset) {
   return GDR_OK;
 }
 
-GDR_API int gdr_abi_version(void) { return 3; }
+GDR_API int gdr_last_launch(gdr_launch_info* info) {
+  if (info == nullptr) return fail(GDR_ERR_NULL, "info is NULL");
+  *info = g_last_launch;
+  return GDR_OK;
+}
+
+GDR_API int gdr_kernel_form_count(void) { return static_cast<int>(kernel_forms().size()); }
+
+GDR_API int gdr_kernel_form(int i, gdr_launch_info* info) {
+  if (info == nullptr) return fail(GDR_ERR_NULL, "info is NULL");
+  const std::vector<gdr_launch_info> forms = kernel_forms();
+  if (i < 0 || i >= static_cast<int>(forms.size()))
+    return fail(GDR_ERR_DIMS, "kernel form index out of range");
+  *info = forms[i];
+  return GDR_OK;
+}
+
+GDR_API int gdr_abi_version(void) { return 5; }
+
+#ifdef GDR_TEST_HOOKS
+// Test builds only (libgdr_testhooks.so): shorten the budget of the
+// abandonable waits (cycles; <= 0 restores the shipped ~2 s) and hold back the
+// tile with index `hold_tile` (< 0: none) in every decode kernel. Synchronous.
+// Not part of the library's ABI: the shipped libgdr.so does not contain it.
+GDR_API int gdrtest_set_hooks(long long wait_limit_cycles, int hold_tile) {
+  const long long limit = wait_limit_cycles > 0 ? wait_limit_cycles : gdr::kWaitLimitCycles;
+  cudaError_t err = cudaMemcpyToSymbol(gdr::g_test_wait_limit, &limit, sizeof(limit));
+  if (err == cudaSuccess)
+    err = cudaMemcpyToSymbol(gdr::g_test_hold_tile, &hold_tile, sizeof(hold_tile));
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("setting the test hooks: ") + cudaGetErrorString(err));
+  return GDR_OK;
+}
+#endif
 
 }  // extern "C"

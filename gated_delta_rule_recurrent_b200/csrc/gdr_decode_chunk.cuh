@@ -149,7 +149,7 @@ __host__ __device__ inline int chunk_stage_bytes(int T) {
 template <int DK, int VS>
 __host__ __device__ inline int chunk_smem_bytes(int T, int n_stages) {
   return 1024 /* alignment slack */ + n_stages * chunk_stage_bytes<DK, VS>(T) +
-         kChunkBarriers * n_stages * 8;
+         kChunkBarriers * n_stages * 8 + 16 /* the abort word (gdr_ptx.cuh) */;
 }
 
 // In-register butterfly reduce-scatter of N values (N a power of two) over the
@@ -718,6 +718,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
   const uint32_t sta0 = vec0 + 8 * n_stages;    // state tile landed
   const uint32_t full0 = sta0 + 8 * n_stages;   // tile finalised (in tile order)
   const uint32_t empty0 = full0 + 8 * n_stages; // the group is done with the stage
+  volatile int* abort_word = reinterpret_cast<volatile int*>(bars + 4 * n_stages);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -736,6 +737,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       mbar_init(full0 + 8 * i, NF);    // one arrival per finaliser warp
       mbar_init(empty0 + 8 * i, CWT);  // one arrival per warp of the group
     }
+    *abort_word = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -745,15 +747,20 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     // Every tile in tile order: wait for its vectors (not for the state),
     // compute the gate and this warp's rows of u, w, e, c and partial sums of
     // A and B, and mark the tile finalised.
+    // A finaliser that saw a wait fail signals no tile ready again, but keeps
+    // meeting the other finaliser on the named barrier every tile.
     const int fw = warp - first_finalizer;
+    bool dead = false;
     for (int j = 0; j < n_mine; ++j) {
       const int tile = blockIdx.x + j * gridDim.x;
       const int h = (tile / n_slices) % p.H_v;
       const int b = tile / (n_slices * p.H_v);
       const int stage = j % n_stages;
       uint8_t* vb = vec_base + stage * lay.bytes;
-      if (!mbar_wait_bounded(vec0 + 8 * stage, (j / n_stages) & 1)) flag_error(kErrProducerWait);
-      int L = reinterpret_cast<const int*>(vb + lay.meta)[0];
+      const bool landed = !dead && mbar_wait_abandonable(vec0 + 8 * stage, (j / n_stages) & 1,
+                                                         abort_word, kErrProducerWait);
+      dead = !__all_sync(0xffffffffu, landed);
+      int L = dead ? 0 : reinterpret_cast<const int*>(vb + lay.meta)[0];
       L = L < 0 ? 0 : (L > T ? T : L);
       const int n_commit = reinterpret_cast<const int*>(vb + lay.meta)[2];
       if (L > 0) {
@@ -779,15 +786,13 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       named_barrier(1, 32 * NF);  // every finaliser takes the same path: no early exits
       if (L > 0) chunk_sum_parts<NF>(vb, lay, L, lane, fw);
       __syncwarp();
-      if (lane == 0) mbar_arrive(full0 + 8 * stage);
+      if (lane == 0 && !dead) mbar_arrive(full0 + 8 * stage);
     }
-    // (the consumers wait for every state tile, so no copy outlives the CTA)
     return;
   }
 
   if (warp == producer) {
     // ================================================================ producer
-    bool failed = false;
     // lane i holds the slot, length and committed count of tile (j & ~31) + i;
     // the next 32 tiles' are loaded 32 tiles ahead (no committed-count array:
     // every token is committed)
@@ -805,7 +810,14 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
     int cur_s, cur_L, cur_n, nxt_s, nxt_L, nxt_n;
     load_index(lane, cur_s, cur_L, cur_n);
     load_index(32 + lane, nxt_s, nxt_L, nxt_n);
+    // tiles issued: all of them, unless a wait for a free stage fails or (test
+    // builds) a tile is held back; from there on nothing is issued or signalled
+    int n_issue = n_mine;
     for (int j = 0; j < n_mine; ++j) {
+      if (test_hold_tile(blockIdx.x + j * gridDim.x)) {
+        n_issue = j;
+        break;
+      }
       if (j > 0 && (j & 31) == 0) {
         cur_s = nxt_s;
         cur_L = nxt_L;
@@ -827,13 +839,14 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       uint8_t* vb = vec_base + stage * lay.bytes;
       const uint32_t vbar = vec0 + 8 * stage;
       const uint32_t sbar = sta0 + 8 * stage;
-      if (lane == 0 && !failed) {
-        if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1)) {
-          failed = true;
-          flag_error(kErrProducerWait);
-        }
+      bool free_ok = true;
+      if (lane == 0)
+        free_ok = mbar_wait_abandonable(empty0 + 8 * stage, phase ^ 1, abort_word,
+                                        kErrProducerWait);
+      if (!__shfl_sync(0xffffffffu, free_ok, 0)) {
+        n_issue = j;
+        break;
       }
-      __syncwarp();
       if (lane == 0) {
         int* meta = reinterpret_cast<int*>(vb + lay.meta);
         meta[0] = L;
@@ -887,6 +900,16 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       }
       cp_async_arrive_noinc(vbar);
     }
+    // No copy may outlive the CTA: wait (bounded, not abandonable) for both
+    // barriers of the last tile issued into every stage.
+    for (int k = (n_issue > n_stages ? n_issue - n_stages : 0); k < n_issue; ++k) {
+      const uint32_t ph = (k / n_stages) & 1;
+      if (!mbar_wait_bounded(vec0 + 8 * (k % n_stages), ph) ||
+          !mbar_wait_bounded(sta0 + 8 * (k % n_stages), ph)) {
+        if (lane == 0) flag_error(kErrDrainWait);
+        break;
+      }
+    }
     return;
   }
 
@@ -898,6 +921,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
   const int c0 = gw * kChunkWarpCols + (lane & 7) * 4;  // first tile column of this lane
   const int col = c0 + solved_column(rg);               // the column this lane solves
   const int tj = gw * 32 + lane;                        // VK: first row of this thread
+  bool dead = false;  // a wait of this warp failed: it commits and frees nothing more
   for (int it = group; it < n_mine; it += n_groups) {
     const int tile = blockIdx.x + it * gridDim.x;
     const int slice = tile % n_slices;
@@ -910,16 +934,18 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
 
     // finalised (in tile order), then the state tile itself: it was issued
     // before the tile was finalised, so its barrier is at this tile's phase
-    bool ok_self = mbar_wait_bounded(full0 + 8 * stage, phase);
-    ok_self = mbar_wait_bounded(sta0 + 8 * stage, phase) && ok_self;
+    bool ok_self =
+        !dead && mbar_wait_abandonable(full0 + 8 * stage, phase, abort_word, kErrConsumerWait);
+    ok_self = ok_self &&
+              mbar_wait_abandonable(sta0 + 8 * stage, phase, abort_word, kErrConsumerWait);
     const bool ok = __all_sync(0xffffffffu, ok_self);
-    if (!ok_self) flag_error(kErrConsumerWait);
+    dead = !ok;
     const int* meta = reinterpret_cast<const int*>(vb + lay.meta);
     int L = ok ? meta[0] : 0;
     L = L < 0 ? 0 : (L > T ? T : L);
     const int s = meta[1];
     if (s < 0 || s >= p.pool_size) L = 0;
-    const bool commit = meta[2] > 0;  // else the slot keeps its bits (pass 2 is skipped)
+    const bool commit = ok && meta[2] > 0;  // else the slot keeps its bits (pass 2 is skipped)
 
     // out[b, h, t, slice * VS + column]; padded tokens get +0.0
     const size_t bh = static_cast<size_t>(b) * p.H_v + h;
@@ -945,7 +971,7 @@ __global__ void __launch_bounds__(kChunkMaxThreads, 1)
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+    if (lane == 0 && !dead) mbar_arrive(empty0 + 8 * stage);
   }
 }
 

@@ -134,7 +134,7 @@ constexpr int kTcGroupBytes = 26624;
 __host__ __device__ inline int tc_smem_bytes(int T, int n_stages, int n_groups) {
   const int vec = (n_stages * tc_layout(T).bytes + 1023) & ~1023;
   return 1024 /* alignment slack */ + n_stages * kTcStateBytes + vec + n_groups * kTcGroupBytes +
-         (4 * n_stages + n_groups) * 8 + 16;
+         (4 * n_stages + n_groups) * 8 + 16 /* TMEM address, abort word (gdr_ptx.cuh) */;
 }
 
 // Eight fp32 values as bf16 (hi, lo) parts, packed in pairs: hi = bf16(x),
@@ -542,6 +542,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
   const uint32_t ab0 = empty0 + 8 * n_stages;     // the stage's A and B are summed (SUMS)
   const uint32_t mma0 = ab0 + 8 * n_stages;       // a group's MMAs are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * n_stages + n_groups);
+  volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -560,6 +561,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       mbar_init(ab0 + 8 * i, 1);    // lane 0 of the group's sums warp (SUMS)
     }
     for (int g = 0; g < n_groups; ++g) mbar_init(mma0 + 8 * g, 1);  // one MMA commit
+    *abort_word = 0;
     fence_mbar_init();
   }
   __syncwarp();
@@ -574,7 +576,6 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
 
   if (warp == producer) {
     // ================================================================ producer
-    bool failed = false;
     // lane i holds the slot, length and committed count of tile (j & ~31) + i;
     // the next 32 tiles' are loaded 32 tiles ahead
     auto load_index = [&](int jj, int& slot, int& len, int& acc) {
@@ -591,7 +592,14 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     int cur_s, cur_L, cur_n, nxt_s, nxt_L, nxt_n;
     load_index(lane, cur_s, cur_L, cur_n);
     load_index(32 + lane, nxt_s, nxt_L, nxt_n);
+    // tiles issued: all of them, unless a wait for a free stage fails or (test
+    // builds) a tile is held back; from there on nothing is issued or signalled
+    int n_issue = n_mine;
     for (int j = 0; j < n_mine; ++j) {
+      if (test_hold_tile(blockIdx.x + j * gridDim.x)) {
+        n_issue = j;
+        break;
+      }
       if (j > 0 && (j & 31) == 0) {
         cur_s = nxt_s;
         cur_L = nxt_L;
@@ -613,13 +621,14 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       uint8_t* vb = vec_base + stage * lay.bytes;
       const uint32_t vbar = vec0 + 8 * stage;
       const uint32_t sbar = sta0 + 8 * stage;
-      if (lane == 0 && !failed) {
-        if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1)) {
-          failed = true;
-          flag_error(kErrProducerWait);
-        }
+      bool free_ok = true;
+      if (lane == 0)
+        free_ok = mbar_wait_abandonable(empty0 + 8 * stage, phase ^ 1, abort_word,
+                                        kErrProducerWait);
+      if (!__shfl_sync(0xffffffffu, free_ok, 0)) {
+        n_issue = j;
+        break;
       }
-      __syncwarp();
       if (lane == 0) {
         int* meta = reinterpret_cast<int*>(vb + lay.meta);
         meta[0] = L;
@@ -673,16 +682,32 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       }
       cp_async_arrive_noinc(vbar);
     }
+    // No copy may outlive the CTA: wait (bounded, not abandonable) for both
+    // barriers of the last tile issued into every stage (the last n_stages
+    // tiles issued fill each stage once).
+    for (int k = (n_issue > n_stages ? n_issue - n_stages : 0); k < n_issue; ++k) {
+      const int stg = tc_stage(k, n_groups, per_group);
+      const uint32_t ph = tc_phase(k, n_groups, per_group);
+      if (!mbar_wait_bounded(vec0 + 8 * stg, ph) || !mbar_wait_bounded(sta0 + 8 * stg, ph)) {
+        if (lane == 0) flag_error(kErrDrainWait);
+        break;
+      }
+    }
   } else if (SUMS && warp >= first_sums) {
     // ================================================================ the L x L sums
-    for (int j = warp - first_sums; j < n_mine; j += n_groups) {
+    bool dead = false;  // a wait failed: this warp signals no tile ready again
+    for (int j = warp - first_sums; j < n_mine && !dead; j += n_groups) {
       const int tile = blockIdx.x + j * gridDim.x;
       const int h = (tile / n_slices) % p.H_v;
       const int b = tile / (n_slices * p.H_v);
       const int stage = tc_stage(j, n_groups, per_group);
       const uint8_t* vb = vec_base + stage * lay.bytes;
-      if (!mbar_wait_bounded(vec0 + 8 * stage, tc_phase(j, n_groups, per_group)))
-        flag_error(kErrProducerWait);
+      const bool landed = mbar_wait_abandonable(vec0 + 8 * stage, tc_phase(j, n_groups, per_group),
+                                                abort_word, kErrProducerWait);
+      if (!__all_sync(0xffffffffu, landed)) {
+        dead = true;
+        break;
+      }
       int L = reinterpret_cast<const int*>(vb + lay.meta)[0];
       L = L < 0 ? 0 : (L > T ? T : L);
       if (L > 0) {
@@ -726,6 +751,9 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     constexpr uint32_t idesc2 = umma_idesc_bf16<kTcDK, kTcVS, false, false>();
     uint32_t mma_phase = 0;
     int held = -1;  // the stage whose new state is still being stored (elected thread)
+    // A wait of the group failed (decided by a vote, so the whole group agrees):
+    // from then on it commits no state and frees no stage.
+    bool dead = false;
 
     for (int it = group; it < n_mine; it += n_groups) {
       const int tile = blockIdx.x + it * gridDim.x;
@@ -737,9 +765,11 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       uint8_t* st = smem + stage * kTcStateBytes;
       const uint8_t* vb = vec_base + stage * lay.bytes;
 
-      bool ok_self = mbar_wait_bounded(vec0 + 8 * stage, phase);
+      bool ok_self =
+          !dead && mbar_wait_abandonable(vec0 + 8 * stage, phase, abort_word, kErrConsumerWait);
       const int* meta = reinterpret_cast<const int*>(vb + lay.meta);
-      int L = meta[0];
+      // one value per warp (the finalise below shuffles); 0 where a lane's wait failed
+      int L = __all_sync(0xffffffffu, ok_self) ? meta[0] : 0;
       L = L < 0 ? 0 : (L > T ? T : L);
       const int s = meta[1];
       if (s < 0 || s >= p.pool_size) L = 0;
@@ -775,13 +805,18 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       fence_async_smem();
       if (elected && held >= 0) {  // the previous tile's store has read its stage by now
         bulk_wait_read_all();
-        mbar_arrive(empty0 + 8 * held);
+        if (!dead) mbar_arrive(empty0 + 8 * held);
         held = -1;
       }
-      ok_self = mbar_wait_bounded(sta0 + 8 * stage, phase) && ok_self;
-      if (!ok_self) flag_error(kErrConsumerWait);
+      ok_self = ok_self &&
+                mbar_wait_abandonable(sta0 + 8 * stage, phase, abort_word, kErrConsumerWait);
       tc_fence_before();
-      named_barrier(bar_id, kTcGroupThreads);  // operands and slots written; D1 free
+      // operands and slots written; D1 free. The vote: the tile goes on only if
+      // every thread of the group saw both its copies land.
+      if (!named_barrier_and(bar_id, kTcGroupThreads, ok_self)) {
+        dead = true;
+        L = 0;
+      }
 
       // ---- 2. pass 1 on the tensor cores; A and B on the CUDA cores
       if (L > 0) {
@@ -806,10 +841,13 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         }
         if constexpr (!SUMS) tc_sum_parts(gb, L, r);
       }
+      bool sums_ok = true;
       if constexpr (SUMS) {
         // A and B from the sums warp (waited for every tile, so that no later
         // wait on this stage can see a phase two fills old)
-        if (!mbar_wait_bounded(ab0 + 8 * stage, phase)) flag_error(kErrConsumerWait);
+        sums_ok = !dead &&
+                  mbar_wait_abandonable(ab0 + 8 * stage, phase, abort_word, kErrConsumerWait);
+        sums_ok = __all_sync(0xffffffffu, sums_ok);  // one decision per warp (the solve shuffles)
       } else {
         named_barrier(bar_id, kTcGroupThreads);  // A and B ready
       }
@@ -825,14 +863,16 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         const float* sa = SUMS ? reinterpret_cast<const float*>(vb + lay.ab)
                                : reinterpret_cast<const float*>(gb + kTcA);
         const float* sb = SUMS ? sa + 64 : reinterpret_cast<const float*>(gb + kTcBm);
-        tc_solve_any(L, x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
+        if (sums_ok) tc_solve_any(L, x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
       }
       fence_async_smem();
       tc_fence_before();
-      named_barrier(bar_id, kTcGroupThreads);  // delta operand written; D1 reads done
+      // delta operand written; D1 reads done. The vote: commit only if every
+      // warp of the group had its A and B.
+      if (!named_barrier_and(bar_id, kTcGroupThreads, sums_ok)) dead = true;
 
       // ---- 4. pass 2 and the new state, when any token is committed
-      const bool commit = L > 0 && n_commit > 0;  // else the slot keeps its bits
+      const bool commit = L > 0 && n_commit > 0 && !dead;  // else the slot keeps its bits
       if (commit) {
         if (wq == 0) {
           if (elect_one()) {
@@ -874,7 +914,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     if (elected) {
       if (held >= 0) {
         bulk_wait_read_all();
-        mbar_arrive(empty0 + 8 * held);
+        if (!dead) mbar_arrive(empty0 + 8 * held);
       }
       bulk_wait_all();
     }

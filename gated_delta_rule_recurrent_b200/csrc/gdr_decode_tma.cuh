@@ -131,8 +131,9 @@ __host__ __device__ inline StageLayout stage_layout(int T) {
   return s;
 }
 
-// CTA-level area after the stages: three mbarriers per stage.
-__host__ __device__ inline int cta_extra_bytes(int n_stages) { return 3 * n_stages * 8; }
+// CTA-level area after the stages: three mbarriers per stage, then the abort
+// word of the failure protocol (gdr_ptx.cuh).
+__host__ __device__ inline int cta_extra_bytes(int n_stages) { return 3 * n_stages * 8 + 16; }
 
 template <int DK, int VS, int R>
 __host__ __device__ inline int tma_smem_bytes(int T, int n_stages) {
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
   const uint32_t raw0 = smem_addr(bars);         // copies landed
   const uint32_t full0 = raw0 + 8 * n_stages;    // producer finished the stage
   const uint32_t empty0 = full0 + 8 * n_stages;  // consumers are done reading the stage
+  volatile int* abort_word = reinterpret_cast<volatile int*>(bars + 3 * n_stages);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -181,6 +183,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, CW);  // one arrival per consumer warp
     }
+    *abort_word = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -188,7 +191,11 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
   if (warp == CW) {
     // ================================================================ producer
     constexpr int E = DK / 32;  // row elements per lane in the finalise step
-    bool failed = false;
+    // Tiles this warp issues: all of them, unless a wait fails (then it stops
+    // issuing and signals nothing more) or, in a test build, a tile is held back
+    // (then it stops issuing but still finalises the tiles already issued).
+    int n_issue = n_mine;
+    bool silent = false;
     // slot, length and committed count of the next tile to issue, loaded one
     // iteration ahead (no committed-count array: all tokens are committed)
     int nx_s = 0, nx_L = 0, nx_n = 0;
@@ -198,8 +205,9 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
       nx_L = p.seq_lengths[b0];
       nx_n = p.num_accepted != nullptr ? p.num_accepted[b0] : T;
     }
-    for (int j = 0; j < n_mine + kLookahead; ++j) {
-      if (j < n_mine) {
+    for (int j = 0; j < n_issue + kLookahead && !silent; ++j) {
+      if (j < n_issue && test_hold_tile(blockIdx.x + j * gridDim.x)) n_issue = j;
+      if (j < n_issue) {
         // ---- issue tile j: start every copy it needs
         const int tile = blockIdx.x + j * gridDim.x;
         const int slice = tile % n_slices;
@@ -220,13 +228,15 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         const uint32_t phase = (j / n_stages) & 1;
         uint8_t* st = smem + stage * lay.bytes;
         const uint32_t rawb = raw0 + 8 * stage;
-        if (lane == 0 && !failed) {
-          if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1)) {
-            failed = true;
-            flag_error(kErrProducerWait);
-          }
+        bool free_ok = true;
+        if (lane == 0)
+          free_ok = mbar_wait_abandonable(empty0 + 8 * stage, phase ^ 1, abort_word,
+                                          kErrProducerWait);
+        if (!__shfl_sync(0xffffffffu, free_ok, 0)) {
+          silent = true;  // the stage may still be in use: start nothing more
+          n_issue = j;
+          break;
         }
-        __syncwarp();
         const int col0 = slice * VS;
         const int hq = h / p.group;
         if (lane == 0) {
@@ -273,7 +283,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         }
         cp_async_arrive_noinc(rawb);
       }
-      if (j >= kLookahead) {
+      if (j >= kLookahead && j - kLookahead < n_issue) {
         // ---- finalise tile j - kLookahead: its copies have landed
         const int jf = j - kLookahead;
         const int tile = blockIdx.x + jf * gridDim.x;
@@ -282,7 +292,12 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
         const int stage = jf % n_stages;
         const uint32_t phase = (jf / n_stages) & 1;
         uint8_t* st = smem + stage * lay.bytes;
-        if (!mbar_wait_bounded(raw0 + 8 * stage, phase)) flag_error(kErrProducerWait);
+        const bool landed = mbar_wait_abandonable(raw0 + 8 * stage, phase, abort_word,
+                                                  kErrProducerWait);
+        if (!__all_sync(0xffffffffu, landed)) {
+          silent = true;  // copies not seen to land: this tile is never signalled ready
+          break;
+        }
         int L = reinterpret_cast<const int*>(st + lay.meta)[0];
         L = L < 0 ? 0 : (L > T ? T : L);
         const uint32_t* rawv = reinterpret_cast<const uint32_t*>(st + lay.raw);
@@ -342,8 +357,9 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
       }
     }
     // Before the CTA may retire, the copies this warp started must have landed:
-    // wait (bounded) for the last raw phase of every stage still in use.
-    for (int k = (n_mine > n_stages ? n_mine - n_stages : 0); k < n_mine; ++k) {
+    // wait (bounded, not abandonable) for the raw phase of the last tile issued
+    // into every stage.
+    for (int k = (n_issue > n_stages ? n_issue - n_stages : 0); k < n_issue; ++k) {
       if (!mbar_wait_bounded(raw0 + 8 * (k % n_stages), (k / n_stages) & 1)) {
         flag_error(kErrDrainWait);
         break;
@@ -367,6 +383,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
   const bool b4 = (lane >> 4) & 1;
   const int cred = cg * 8 + NV * (rl & (RL / 2 - 1));
 
+  bool dead = false;  // a wait of this warp failed: it commits and frees nothing more
   for (int it = 0; it < n_mine; ++it) {
     const int tile = blockIdx.x + it * gridDim.x;
     const int slice = tile % n_slices;
@@ -376,16 +393,17 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     const uint32_t phase = (it / n_stages) & 1;
     uint8_t* st = smem + stage * lay.bytes;
 
-    const bool ok_self = mbar_wait_bounded(full0 + 8 * stage, phase);
+    const bool ok_self =
+        !dead && mbar_wait_abandonable(full0 + 8 * stage, phase, abort_word, kErrConsumerWait);
     const bool ok = __all_sync(0xffffffffu, ok_self);
-    if (!ok_self) flag_error(kErrConsumerWait);
+    dead = !ok;
     const int* meta = reinterpret_cast<const int*>(st + lay.meta);
     int L = ok ? meta[0] : 0;  // one load for the whole warp: every lane sees one value
     L = L < 0 ? 0 : (L > T ? T : L);
     L = L > 1 ? 1 : L;  // single-token calls
     const int s = meta[1];
     if (s < 0 || s >= p.pool_size) L = 0;
-    const bool commit = meta[2] > 0;  // else the call leaves the slot's bits as they are
+    const bool commit = ok && meta[2] > 0;  // else the call leaves the slot's bits as they are
 
     // out[b, h, :, slice * VS + cband : + WCOLS]; padded tokens get +0.0.
     uint16_t* out_band =
@@ -549,7 +567,7 @@ __global__ void __launch_bounds__(TmaShape<DK, VS, RR>::kThreads, 1)
     }
     // This warp has read everything it needs from the stage: give it back.
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+    if (lane == 0 && !dead) mbar_arrive(empty0 + 8 * stage);
   }
 }
 

@@ -22,6 +22,26 @@ static __device__ unsigned int g_device_error = 0;
 
 constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
+// Test builds only (-DGDR_TEST_HOOKS, never the shipped library): the limit of
+// the abandonable waits below is a device variable the host can shorten, and
+// the producer of every decode kernel can hold back one tile: it then starts
+// no copy for that tile and never signals it ready, as if its copies never
+// landed, and stops issuing. Its consumers' waits run out, with no copy in
+// flight anywhere.
+#ifdef GDR_TEST_HOOKS
+static __device__ long long g_test_wait_limit = kWaitLimitCycles;
+static __device__ int g_test_hold_tile = -1;
+__device__ __forceinline__ long long abandonable_wait_limit() {
+  return *reinterpret_cast<volatile long long*>(&g_test_wait_limit);
+}
+__device__ __forceinline__ bool test_hold_tile(int tile) {
+  return tile == *reinterpret_cast<volatile int*>(&g_test_hold_tile);
+}
+#else
+__device__ __forceinline__ constexpr long long abandonable_wait_limit() { return kWaitLimitCycles; }
+__device__ __forceinline__ constexpr bool test_hold_tile(int) { return false; }
+#endif
+
 // Byte offset of (row i, 16-byte chunk holding column col) in a state tile
 // loaded by TMA with the 128-byte swizzle as [col / 64][row][64 columns]:
 // within each 128-byte row segment, chunk c sits at position c ^ (i % 8).
@@ -82,7 +102,9 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 constexpr uint32_t kWaitSuspendNs = 20000;
 
 // Wait for the phase of parity `parity` to complete, for at most
-// kWaitLimitCycles. Returns false when the budget ran out.
+// kWaitLimitCycles. Returns false when the budget ran out. Used for work that
+// is already in flight and ends by itself: copies a CTA must see land before
+// it exits, and tensor-core MMAs it issued.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -90,6 +112,49 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
   return true;
+}
+
+// Failure protocol of the decode kernels. Each CTA keeps an abort word in
+// shared memory (0 at start). A wait on another role's signal ("ready",
+// "free") is abandonable: it returns false when its own budget runs out (it
+// then ORs `err_bit` into the device error word and sets the abort word), or,
+// once it has to block, as soon as the abort word is set by any other wait of
+// the CTA. Whoever sees a wait fail stops for good: a producer issues no more
+// copies, a finaliser or sums warp signals no more tiles ready, a consumer
+// commits no state and frees no more stages. Because nobody signals after a
+// failure, no stage is refilled over a phase that never completed, so no wait
+// can mistake an old phase for a new one; the tiles a CTA commits are exactly
+// the ones whose inputs were seen to land. Copies already started are drained
+// with mbar_wait_bounded before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_abandonable(uint32_t bar, uint32_t parity,
+                                                      volatile int* abort_word, unsigned err_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long limit = abandonable_wait_limit();
+  const long long t0 = clock64();
+  while (!mbar_try_wait_suspend(bar, parity, kWaitSuspendNs)) {
+    if (*abort_word != 0) return false;
+    if (clock64() - t0 > limit) {
+      atomicOr(&g_device_error, err_bit);
+      *abort_word = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// bar.sync over `count` threads that also ANDs a predicate across them: every
+// participant gets true exactly when every participant passed true.
+__device__ __forceinline__ bool named_barrier_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,

@@ -159,6 +159,51 @@ GDR_API int gdr_gate_fused(const gdr_dims* dims, const gdr_bf16* query, const gd
                            const float* gk, const int32_t* num_accepted_tokens,
                            float scale_value, gdr_bf16* out, gdr_stream_t stream);
 
+/*
+ * gdr_prefill - the op's recurrence over a long prompt: the four steps of
+ * "lite_boost.ops.recurrent_gated_delta_rule" (section 算法流程) for every
+ * valid token, in token order. The page's op is decode-only and sends prefill
+ * to a chunk-level op (section 注); this entry point computes the same
+ * result for any token count, with the arguments of gdr_decode.
+ *
+ * Arguments, layouts, ownership and the treatment of lengths, slots and
+ * committed counts are those of gdr_decode, except:
+ *   T                   any T >= 1 (the padded token count of the call);
+ *   sizes               D_k = 128, D_v a multiple of 128, dims->layout =
+ *                       GDR_LAYOUT_KV; other sizes return GDR_ERR_UNSUPPORTED;
+ *   precision           the state is carried in fp32 across all L valid tokens
+ *                       of an item and rounded to bf16 once, as in gdr_decode;
+ *                       inside a chunk of 8 tokens the tensor-core products
+ *                       read the state as bf16 hi + lo parts (16 significant
+ *                       bits) and the per-token vectors likewise;
+ *   num_accepted_tokens as for gdr_decode: the slot receives the state after
+ *                       the first n tokens, the outputs of all L tokens are
+ *                       computed.
+ * Tensor memory: a launch takes all 512 columns of each SM it runs on for its
+ * duration (see gdr_decode's kernels: one CTA per SM, freed before exit), so
+ * it must not share an SM with another kernel that holds tensor memory.
+ * Returns a gdr_status.
+ */
+GDR_API int gdr_prefill(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
+                        const gdr_bf16* value, const gdr_bf16* beta, gdr_bf16* state_pool,
+                        const int32_t* actual_seq_lengths, const int32_t* ssm_state_indices,
+                        const float* g, const float* gk, const int32_t* num_accepted_tokens,
+                        float scale_value, gdr_bf16* out, gdr_stream_t stream);
+
+/*
+ * gdr_prefill_gated - gdr_prefill with the LinearAttentionGate computed in
+ * the kernel, as for gdr_gate_fused ("com.microsoft.LinearAttentionGate",
+ * section Description): a, b [B, T, H_v] bf16, dt_bias and decay_scale [H_v]
+ * fp32 in place of g and beta. Returns a gdr_status.
+ */
+GDR_API int gdr_prefill_gated(const gdr_dims* dims, const gdr_bf16* query, const gdr_bf16* key,
+                              const gdr_bf16* value, const gdr_bf16* a, const gdr_bf16* b,
+                              const float* dt_bias, const float* decay_scale,
+                              gdr_bf16* state_pool, const int32_t* actual_seq_lengths,
+                              const int32_t* ssm_state_indices, const float* gk,
+                              const int32_t* num_accepted_tokens, float scale_value,
+                              gdr_bf16* out, gdr_stream_t stream);
+
 /* Element types of the standalone gate's a, b, decay and beta. */
 typedef enum gdr_dtype {
   GDR_DTYPE_F32 = 0,  /* float32, one of the gate page's types (Type constraints) */
@@ -216,8 +261,49 @@ GDR_API const char* gdr_last_error(void);
  * counterpart on the pages: every bounded wait of the kernels reports here. */
 GDR_API int gdr_device_error(uint32_t* flags, int reset);
 
-/* Library ABI version, currently 3 (2 added gdr_linear_attention_gate, 3 the
- * layout field of gdr_dims). */
+/* Kernel families of the library (gdr_launch_info.kernel). */
+typedef enum gdr_kernel {
+  GDR_KERNEL_NONE = 0,
+  GDR_KERNEL_SINGLE_TOKEN = 1,     /* one token per call, CUDA cores */
+  GDR_KERNEL_CHUNKED = 2,          /* several tokens (or a k-contiguous pool), CUDA cores */
+  GDR_KERNEL_TENSOR_CORE = 3,      /* D_k = 128, D_v a multiple of 128, several tokens */
+  GDR_KERNEL_TENSOR_CORE_ONE = 4,  /* the same kernel's form for one token per call */
+  GDR_KERNEL_GATE = 5,             /* the standalone gate */
+  GDR_KERNEL_PREFILL = 6           /* gdr_prefill / gdr_prefill_gated */
+} gdr_kernel;
+
+/* One kernel launch: its family, the key width, the column width of a tile
+ * (0 for the gate), whether the gate is fused, the pool layout, and the launch
+ * shape (blocks, threads per block, dynamic shared memory, pipeline stages). */
+typedef struct gdr_launch_info {
+  int32_t kernel;
+  int32_t D_k;
+  int32_t tile_cols;
+  int32_t gated;
+  int32_t layout;
+  int32_t grid;
+  int32_t threads;
+  int32_t smem_bytes;
+  int32_t stages;
+} gdr_launch_info;
+
+/* The most recent kernel launch the calling thread made through the library
+ * (kernel = GDR_KERNEL_NONE before the first one, and for a call that queued
+ * nothing, such as B = 0). Host-only; no counterpart on the pages: it lets a
+ * caller or a test see which kernel and tile width the dispatcher chose.
+ * Returns GDR_ERR_NULL for a NULL `info`, else GDR_OK. */
+GDR_API int gdr_last_launch(gdr_launch_info* info);
+
+/* The decode kernel forms the dispatcher can choose, as (kernel, D_k,
+ * tile_cols, gated, layout); the launch-shape fields are 0. gdr_kernel_form
+ * fills form `i`, 0 <= i < gdr_kernel_form_count(), and returns GDR_ERR_DIMS
+ * for any other i. Host-only, needs no GPU; no counterpart on the pages. */
+GDR_API int gdr_kernel_form_count(void);
+GDR_API int gdr_kernel_form(int i, gdr_launch_info* info);
+
+/* Library ABI version, currently 5 (2 added gdr_linear_attention_gate, 3 the
+ * layout field of gdr_dims, 4 gdr_last_launch and the kernel forms, 5
+ * gdr_prefill and gdr_prefill_gated). */
 GDR_API int gdr_abi_version(void);
 
 #ifdef __cplusplus

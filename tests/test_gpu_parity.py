@@ -52,6 +52,13 @@ def test_large_batch_gated_full_size_sampled():
     _roundtrip(x, True, items)
 
 
+@pytest.mark.slow
+def test_large_batch_gated_full_size_all_items():
+    """The same call with every one of the 512 items checked against the oracle
+    (about 40 s of oracle time)."""
+    _roundtrip(workloads.make_inputs(4), True)
+
+
 @pytest.mark.parametrize("D_k,D_v,H_qk,H_v,T", [
     (64, 192, 3, 6, 3),     # three column slices, grouped heads
     (128, 320, 2, 8, 5),    # five slices, 4 value heads per q/k head

@@ -199,6 +199,31 @@ def test_tokens_compose():
     np.testing.assert_allclose(st, st_all, rtol=1e-12, atol=1e-14)
 
 
+def test_long_prompt_equals_chunks_of_eight():
+    """A prefill-length call: without rounding, one call over T = 128 tokens
+    equals sixteen consecutive T = 8 calls (the state of each passed to the
+    next), bit for bit, with ragged lengths that end inside a chunk."""
+    c = _rand_case(16, B=3, H_qk=1, H_v=2, T=128, D_k=5, D_v=3, P=4)
+    c["actual_seq_lengths"] = np.array([128, 77, 8])
+    out_all, st_all = _run(c, round_out=False, round_state=False)
+    st = c["state"].copy()
+    for k in range(16):
+        ck = dict(c)
+        sl = slice(8 * k, 8 * k + 8)
+        for name in ("query", "key", "value"):
+            ck[name] = c[name][:, :, sl]
+        for name in ("beta", "g", "gk"):
+            ck[name] = c[name][:, :, sl]
+        ck["actual_seq_lengths"] = np.clip(c["actual_seq_lengths"] - 8 * k, 0, 8)
+        ck["num_accepted_tokens"] = ck["actual_seq_lengths"]
+        ck["state"] = st
+        out_k, st = _run(ck, round_out=False, round_state=False)
+        valid = (8 * k + np.arange(8))[None, :] < c["actual_seq_lengths"][:, None]  # [B, 8]
+        assert np.array_equal(out_k[valid[:, None, :].repeat(2, 1)],
+                              out_all[:, :, sl][valid[:, None, :].repeat(2, 1)])
+    assert np.array_equal(st, st_all)
+
+
 def test_untouched_slots_and_permutation():
     """Slots no item references keep their exact bits; permuting items permutes outputs."""
     c = _rand_case(7, B=3, P=6)
