@@ -40,6 +40,7 @@ if ROOT not in sys.path:
 from gated_delta_rule_recurrent_b200 import distributed, metrics, workloads  # noqa: E402
 
 METRIC = "decode tokens/s and achieved HBM GB/s vs ~8 TB/s peak for gated-delta step"
+PREFILL_METRIC = "prefill tokens/s and achieved HBM GB/s (long-prompt gated-delta recurrence)"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
@@ -302,18 +303,37 @@ def _place(x, dev, layout):
     return xd
 
 
-def _timed_region(step, K, stream, dev, barrier, max_over_ranks):
+def _capture(step, K, dev):
+    """The K steps captured once as a CUDA graph (the library's per-call host
+    work, configuration and tensor maps, happens at capture; a replay queues
+    only the K kernel launches)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(g, stream=s):
+        for i in range(K):
+            step(i)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize(dev)
+    return g
+
+
+def _timed_region(step, K, stream, dev, barrier, max_over_ranks, graph=None):
     """K steps back to back between two events on the launching stream,
-    bracketed by a barrier and a device synchronisation on both sides; the
-    max over ranks of the region, and the host times of its ends."""
+    bracketed by a barrier and a device synchronisation on both sides (as one
+    replay of ``graph`` when given); the max over ranks of the region, and the
+    host times of its ends."""
     r0 = torch.cuda.Event(enable_timing=True)
     r1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     host_t0 = time.time()
     r0.record(stream)
-    for i in range(K):
-        step(i)
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(K):
+            step(i)
     r1.record(stream)
     torch.cuda.synchronize(dev)
     host_t1 = time.time()
@@ -321,8 +341,9 @@ def _timed_region(step, K, stream, dev, barrier, max_over_ranks):
     return max_over_ranks(r0.elapsed_time(r1)), host_t0, host_t1
 
 
-def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
-    """One JSON line for one decode workload on this rank's GPU."""
+def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds, op="decode"):
+    """One JSON line for one decode (or, op="prefill", long-prompt) workload on
+    this rank's GPU."""
     import gated_delta_rule_recurrent_b200 as gdr
 
     world, rank, dev, barrier, max_over_ranks, sampler = ctx
@@ -348,7 +369,17 @@ def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
     stream = torch.cuda.current_stream(dev)
 
     def call(z, o):
-        if gated:
+        if op == "prefill":
+            if gated:
+                gdr.prefill_gated(z["query"], z["key"], z["value"], z["a"], z["b"],
+                                  z["dt_bias"], z["decay_scale"], z["state_pool"],
+                                  z["actual_seq_lengths"], z["ssm_state_indices"], z["gk"],
+                                  z["num_accepted_tokens"], z["scale_value"], out=o)
+            else:
+                gdr.prefill(z["query"], z["key"], z["value"], z["beta"], z["state_pool"],
+                            z["actual_seq_lengths"], z["ssm_state_indices"], z["g"], z["gk"],
+                            z["num_accepted_tokens"], z["scale_value"], out=o)
+        elif gated:
             gdr.decode_gated(z["query"], z["key"], z["value"], z["a"], z["b"],
                              z["dt_bias"], z["decay_scale"], z["state_pool"],
                              z["actual_seq_lengths"], z["ssm_state_indices"], z["gk"],
@@ -374,11 +405,17 @@ def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
     # launch per step, so the average launch duration is the region over the
     # launches. (An event pair around every launch leaves the device idle for
     # a few microseconds between launches, which a short step would count.)
-    region_ms, host_t0, host_t1 = _timed_region(step, K, stream, dev, barrier, max_over_ranks)
+    # The steps are replayed from a CUDA graph: a small step is shorter than the
+    # ~25 us the Python binding takes to queue a call, and a graph is how a
+    # serving loop issues it. (--no-graph times direct calls instead.)
+    graph = None if args.no_graph else _capture(step, K, dev)
+    region_ms, host_t0, host_t1 = _timed_region(step, K, stream, dev, barrier, max_over_ranks,
+                                                graph)
     clocks = sampler.summary(host_t0, host_t1)
     # the same region again, back to back: its spread shows the run's noise
-    repeats = [_timed_region(step, K, stream, dev, barrier, max_over_ranks)[0] / K
+    repeats = [_timed_region(step, K, stream, dev, barrier, max_over_ranks, graph)[0] / K
                for _ in range(args.repeats)]
+    del graph
     launches = K  # one kernel per step (the decode kernel)
     total_tokens = distributed.sum_over_ranks(n_tokens * K, dev)
     kernel_ms = region_ms / launches
@@ -399,7 +436,8 @@ def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, toks, items, secs = oracle_tokens_per_s(x, gated, items_per_call=8,
+        tps, toks, items, secs = oracle_tokens_per_s(x, gated,
+                                                     items_per_call=1 if op == "prefill" else 8,
                                                      budget_s=cpu_seconds)
         cpu = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": f"{items} of {w.B} batch items ({toks} tokens) of the same "
@@ -415,7 +453,8 @@ def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
           f"inputs and pool ({n_copies * step_bytes / 1e6:.0f} MB, over 3x the "
           f"{L2_BYTES / 2**20:.0f} MiB L2), no flush")
     return {
-        "metric": METRIC,
+        "metric": METRIC if op == "decode" else PREFILL_METRIC,
+        "op": op,
         "value": value,
         "unit": "tokens/s",
         "n_gpus": world,
@@ -436,6 +475,8 @@ def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
             "state_layout": "[pool, H_v, D_k, D_v]" if args.layout == "kv"
                             else "[pool, H_v, D_v, D_k]",
             "l2": l2,
+            "launch": ("one CUDA graph replay of the K steps" if not args.no_graph
+                       else "K direct calls through the Python binding"),
             "parallelism": f"one call of {world} x {w.B} items split by item over {world} "
                            f"rank(s), no collective",
         },
@@ -448,7 +489,8 @@ def bench_decode_workload(args, wkey, ctx, with_e2e, cpu_seconds):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth",
-            "kernel": decode_kernel_name(w, args.layout), "kernel_ms": kernel_ms,
+            "kernel": ("gdr::prefill_tc_kernel" if op == "prefill"
+                       else decode_kernel_name(w, args.layout)), "kernel_ms": kernel_ms,
             "kernel_form": kernel,
             "bytes_per_launch": step_bytes,
             "traffic": recorded_traffic(w.name, args.layout) if n_copies == 1 else None,
@@ -487,8 +529,13 @@ def run_gdr(args):
     sampler = ClockSampler(local, period_ms=10)
     sampler.wait_first()
     ctx = (world, rank, dev, barrier, max_over_ranks, sampler)
-    lines = [bench_decode_workload(args, args.workload, ctx, not args.no_e2e, args.cpu_seconds)]
-    if args.all_workloads:
+    if args.op == "prefill":
+        lines = [bench_decode_workload(args, "prefill", ctx, False, args.cpu_seconds,
+                                       op="prefill")]
+    else:
+        lines = [bench_decode_workload(args, args.workload, ctx, not args.no_e2e,
+                                       args.cpu_seconds)]
+    if args.all_workloads and args.op == "decode":
         for wk in (1, 2, 3):
             if wk != args.workload:
                 lines.append(bench_decode_workload(args, wk, ctx, False,
@@ -644,12 +691,15 @@ def main():
                     help="override B (and the pool size) of the workload, e.g. for a small "
                          "profiling case of the same kernel")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time K direct calls instead of one CUDA-graph replay of them")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
-    ap.add_argument("--op", choices=("decode", "gate"), default="decode",
+    ap.add_argument("--op", choices=("decode", "gate", "prefill"), default="decode",
                     help="decode: the decode step (the default line); gate: the standalone "
-                         "LinearAttentionGate op, a line of its own")
+                         "LinearAttentionGate op; prefill: the long-prompt recurrence "
+                         "(gdr_prefill_gated); each a line of its own")
     ap.add_argument("--gate-shape", default="32768x8x64",
                     help="shape of a and b for --op gate, heads last")
     ap.add_argument("--gate-dtype", choices=("f32", "f16", "bf16"), default="bf16")
@@ -672,6 +722,10 @@ def main():
                                              "see the cpu_baseline key of the gate line"}))
         else:
             run_gate(args)
+    elif args.impl == "reference" and args.op == "prefill":
+        print(json.dumps({"impl": "reference", "op": "prefill",
+                          "unavailable": "the prefill op's reference is the oracle; see the "
+                                         "cpu_baseline key of the prefill line"}))
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -33,7 +33,7 @@ from typing import Dict, Optional, Sequence
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "workload"]
+__all__ = ["Workload", "WORKLOADS", "PREFILL_WORKLOADS", "make_inputs", "workload"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -50,7 +50,7 @@ class Workload:
     pool: int
     scale_value: float
     gated: bool
-    lengths: str  # "full", "fixed" (see fixed_lengths) or "uniform" (U{1..T})
+    lengths: str  # "full", "fixed" (see fixed_lengths), "uniform" (U{1..T}) or "upper" (U{T/2..T})
     indices: str  # "fixed" (see fixed_indices), "subset" (random B of pool) or "perm"
     fixed_lengths: Optional[Sequence[int]] = None
     fixed_indices: Optional[Sequence[int]] = None
@@ -84,13 +84,25 @@ WORKLOADS: Dict[int, Workload] = {
 }
 
 
+# Long-prompt (prefill) workloads: the grouped-head, 128 x 128 shape of the
+# decode workloads over a prompt of up to T tokens, lengths U{T/2..T}, with
+# the fused gate.
+PREFILL_WORKLOADS: Dict[str, Workload] = {
+    "prefill": Workload("prefill_B8_Hqk16_Hv32_T2048_128x128", B=8, H_qk=16, H_v=32, T=2048,
+                        D_k=128, D_v=128, pool=16, scale_value=1.0 / math.sqrt(128),
+                        gated=True, lengths="upper", indices="subset", seed=1005),
+}
+
+
 def workload(key) -> Workload:
     """Look a workload up by number or by name."""
     if isinstance(key, Workload):
         return key
     if isinstance(key, int):
         return WORKLOADS[key]
-    for w in WORKLOADS.values():
+    if key in PREFILL_WORKLOADS:
+        return PREFILL_WORKLOADS[key]
+    for w in list(WORKLOADS.values()) + list(PREFILL_WORKLOADS.values()):
         if w.name == key:
             return w
     raise KeyError(f"unknown workload {key!r}")
@@ -128,6 +140,8 @@ def make_inputs(w, *, seed: Optional[int] = None, poison_padding: bool = False,
         lengths = torch.full((B,), T, dtype=torch.int32)
     elif w.lengths == "uniform":
         lengths = torch.randint(1, T + 1, (B,), generator=gen, dtype=torch.int32)
+    elif w.lengths == "upper":
+        lengths = torch.randint((T + 1) // 2, T + 1, (B,), generator=gen, dtype=torch.int32)
     else:
         raise ValueError(w.lengths)
     if w.indices == "fixed":

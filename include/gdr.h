@@ -49,6 +49,14 @@
  *           check returns its status and queues nothing. GDR_ERR_CUDA reports a
  *           launch failure. gdr_last_error() describes the most recent failure
  *           of the calling thread.
+ * Tensor memory. The kernels for D_k = 128 with D_v a multiple of 128, and the
+ *           prefill kernel, run one CTA per SM and take 512 columns of that
+ *           SM's tensor memory (TMEM) for the length of a launch; they free it
+ *           before they exit. The allocation waits until the columns are free
+ *           (the hardware offers no form that gives up), so a caller must not
+ *           run another kernel that holds TMEM on the same SMs at the same time,
+ *           for example a tcgen05 GEMM on another stream. Calls queued on one
+ *           stream are always safe.
  */
 #ifndef GDR_H_
 #define GDR_H_

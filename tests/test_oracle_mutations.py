@@ -23,6 +23,7 @@ UPD = "S = S + k_t[:, :, None] * delta[:, None, :]"
 
 # (name, [(old, new), ...]) - every `old` must occur in the oracle source.
 MUTATIONS = [
+    ("tokens_capped_at_eight", [("for t in range(L):", "for t in range(min(L, 8)):")]),
     ("decay_without_gk", [(DECAY, "S = S * np.exp(g_t)[:, None, None]")]),
     ("decay_without_g", [(DECAY, "S = S * np.exp(gk[b, :, t, :])[:, :, None]")]),
     ("read_before_decay", [(DECAY, "S_prev = S\n            " + DECAY),
