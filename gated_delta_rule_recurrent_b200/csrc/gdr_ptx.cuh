@@ -118,25 +118,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 // shared memory (0 at start). A wait on another role's signal ("ready",
 // "free") is abandonable: it returns false when its own budget runs out (it
 // then ORs `err_bit` into the device error word and sets the abort word), or,
-// once it has to block, as soon as the abort word is set by any other wait of
-// the CTA. Whoever sees a wait fail stops for good: a producer issues no more
+// once it has blocked for a while, when the abort word is set by any other wait
+// of the CTA. Whoever sees a wait fail stops for good: a producer issues no more
 // copies, a finaliser or sums warp signals no more tiles ready, a consumer
 // commits no state and frees no more stages. Because nobody signals after a
 // failure, no stage is refilled over a phase that never completed, so no wait
 // can mistake an old phase for a new one; the tiles a CTA commits are exactly
 // the ones whose inputs were seen to land. Copies already started are drained
 // with mbar_wait_bounded before the CTA exits.
+//
+// The abort word is looked at only once a wait has lasted a quarter of its
+// budget (never, on a normal call): a wait's loop then costs what a plain
+// bounded wait costs, and a CTA still winds down within a budget of a failure.
 __device__ __forceinline__ bool mbar_wait_abandonable(uint32_t bar, uint32_t parity,
                                                       volatile int* abort_word, unsigned err_bit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long limit = abandonable_wait_limit();
   const long long t0 = clock64();
   while (!mbar_try_wait_suspend(bar, parity, kWaitSuspendNs)) {
-    if (*abort_word != 0) return false;
-    if (clock64() - t0 > limit) {
-      atomicOr(&g_device_error, err_bit);
-      *abort_word = 1;
-      return false;
+    const long long dt = clock64() - t0;
+    if (dt > (limit >> 2)) {
+      if (*abort_word != 0) return false;
+      if (dt > limit) {
+        atomicOr(&g_device_error, err_bit);
+        *abort_word = 1;
+        return false;
+      }
     }
   }
   return true;
