@@ -595,6 +595,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
     // tiles issued: all of them, unless a wait for a free stage fails or (test
     // builds) a tile is held back; from there on nothing is issued or signalled
     int n_issue = n_mine;
+    bool failed = false;  // lane 0: a wait for a free stage ran out (then nothing more)
     for (int j = 0; j < n_mine; ++j) {
       if (test_hold_tile(blockIdx.x + j * gridDim.x)) {
         n_issue = j;
@@ -621,13 +622,12 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
       uint8_t* vb = vec_base + stage * lay.bytes;
       const uint32_t vbar = vec0 + 8 * stage;
       const uint32_t sbar = sta0 + 8 * stage;
-      bool free_ok = true;
-      if (lane == 0)
-        free_ok = mbar_wait_abandonable(empty0 + 8 * stage, phase ^ 1, abort_word,
-                                        kErrProducerWait);
-      if (!__shfl_sync(0xffffffffu, free_ok, 0)) {
-        n_issue = j;
-        break;
+      if (lane == 0 && !failed)
+        failed = !mbar_wait_free(empty0 + 8 * stage, phase ^ 1, abort_word, kErrProducerWait);
+      __syncwarp();
+      if (__shfl_sync(0xffffffffu, failed, 0)) {  // the stage may still be in use
+        if (n_issue == n_mine) n_issue = j;
+        continue;
       }
       if (lane == 0) {
         int* meta = reinterpret_cast<int*>(vb + lay.meta);

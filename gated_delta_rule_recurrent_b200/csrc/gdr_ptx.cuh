@@ -149,6 +149,26 @@ __device__ __forceinline__ bool mbar_wait_abandonable(uint32_t bar, uint32_t par
   return true;
 }
 
+// A producer's wait for a free stage: the loop of mbar_wait_bounded with the
+// budget of the abandonable waits. It does not look at the abort word (a
+// producer waits once per tile, and the extra load in its loop measured ~6 %
+// on the multi-token tensor-core kernel); when the budget runs out it ORs
+// `err_bit` into the device error word, sets the abort word and returns false.
+__device__ __forceinline__ bool mbar_wait_free(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_word, unsigned err_bit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long limit = abandonable_wait_limit();
+  const long long t0 = clock64();
+  while (!mbar_try_wait_suspend(bar, parity, kWaitSuspendNs)) {
+    if (clock64() - t0 > limit) {
+      atomicOr(&g_device_error, err_bit);
+      *abort_word = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
 // bar.sync over `count` threads that also ANDs a predicate across them: every
 // participant gets true exactly when every participant passed true.
 __device__ __forceinline__ bool named_barrier_and(int id, int count, bool pred) {
