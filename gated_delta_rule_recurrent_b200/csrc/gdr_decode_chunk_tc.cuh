@@ -159,11 +159,13 @@ __device__ __forceinline__ void split_bf16x8(const float (&x)[8], uint4& hi, uin
 // and pass-2 operand (e), and, when PAIRS, this warp's partial sums of A and
 // B to slot wq (entry (r, col): B_{t=r, s=col} for col <= r, A_{t=col, s=r}
 // for col > r; without PAIRS a sums warp forms them). The gate value g_t sits
-// in lane t. Returns c_i = P_{n-1}[i] (0 when n = 0).
+// in lane t. Returns c_i = P_{n-1}[i] (0 when n = 0). With nv < LC only the
+// first nv tokens are valid (n <= nv): u and w are zero past them, and the
+// sums that involve a later token are left unspecified (never read).
 template <int LC, bool PAIRS>
 __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& lay, uint8_t* gb,
                                              float g_lane, float scale, int i, int lane, int wq,
-                                             int n) {
+                                             int n, int nv = LC) {
   constexpr int DK = kTcDK;
   constexpr int NM = pow2_at_least(LC * LC);  // partial sums, padded for the reduce-scatter
   float g[LC];
@@ -189,8 +191,10 @@ __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& 
     w[t] = 0.0f;
     if (t < LC) {
       P = t == 0 ? d[0] : P * d[t];
-      u[t] = P * kf[t];
-      w[t] = P * qf[t];
+      if (t < nv) {
+        u[t] = P * kf[t];
+        w[t] = P * qf[t];
+      }
       if (t == n - 1) c = P;
     }
   }
@@ -375,19 +379,20 @@ __device__ __forceinline__ void tc_pair_sums_any(int L, const uint8_t* vb, const
 // Column j of a tile with L = LC tokens, from this thread's TMEM lane of D1:
 // kv_mem and the S_0 part of o per token, the unit lower-triangular solve for
 // delta, o to `out_t0` (token 0, column 0 of the tile's output), and the
-// column's delta row of the pass-2 B operand (zeros past LC). beta_t sits in
-// lane t.
+// column's delta row of the pass-2 B operand (zeros past LC, or past nv when
+// only the first nv tokens are valid). beta_t sits in lane t.
 template <int LC>
 __device__ __forceinline__ void tc_solve(const uint32_t (&x)[32], const uint8_t* vb,
                                          const TcLayout& lay, uint8_t* gb, const float* sa,
                                          const float* sb, float b_lane, int j, uint16_t* out_t0,
-                                         int D_v) {
+                                         int D_v, int nv = LC) {
   const uint16_t* sv = reinterpret_cast<const uint16_t*>(vb + lay.v);
   float dl[8];
 #pragma unroll
   for (int t = 0; t < 8; ++t) dl[t] = 0.0f;
 #pragma unroll
   for (int t = 0; t < LC; ++t) {
+    if (t >= nv) break;  // tokens past nv: no output, delta 0
     const float beta = __shfl_sync(0xffffffffu, b_lane, t);
     // kv_mem_t = S_0^T u_t + sum_{s<t} A_ts delta_s (step 2)
     float kv = __uint_as_float(x[t]) + __uint_as_float(x[8 + t]);

@@ -17,14 +17,21 @@
 //           bf16(S) and S_lo = bf16(S - S_hi), in the TMA's 128-byte swizzled
 //           layout: D1 = S_hi^T [..] + S_lo^T [..], 16 significant bits of S;
 //   solve   per column j: kv_mem, delta (unit lower-triangular), o -> out;
-//   pass 2  S <- c o S + E Delta^T: the TMEM rows are scaled by c (while
-//           pass 1 runs) and pass 2 accumulates into them (tcgen05, M = 128
-//           rows i, N = 128, K = 32);
+//   pass 2  S <- c o S + E Delta^T: the TMEM rows already hold c o S, and
+//           pass 2 accumulates into them (tcgen05, M = 128 rows i, N = 128,
+//           K = 32);
 //   then every thread reads its row of S back and writes S_hi and S_lo for
-//   the next chunk's pass 1. After the chunk that ends at the committed
-//   count n, S_hi is exactly bf16_rne(S_n): the elected thread stores it to
-//   the slot with one TMA store (once per call and tile, as the page's
+//   the next chunk's pass 1, and writes the row back to tensor memory scaled
+//   by the next chunk's c. After the chunk that ends at the committed count
+//   n, S_hi is exactly bf16_rne(S_n): the elected thread stores it to the
+//   slot with one TMA store (once per call and tile, as the page's
 //   state_out; reading D).
+// The consumer loop runs one record behind: the iteration that waits for and
+// finalises chunk k (whose operands depend on the inputs only) then reads
+// back the state chunk k - 1 left, scaling it by chunk k's c on the way, so
+// one group barrier serves both. Chunks run with L = 8 code throughout (a
+// shorter chunk masks the missing tokens), so the finalise and solve are
+// compiled once.
 // Chunks start at multiples of 8 tokens, and one more boundary sits at n when
 // n < L (reading E), so the committed state is the state after token n - 1
 // while outputs continue to token L - 1.
@@ -32,9 +39,11 @@
 // CTA: two consumer groups of four warps (thread r of a group = TMEM lane r =
 // row i in row-wise steps, column j in column-wise ones) and one producer
 // warp per group, one CTA per SM, persistent over tiles; group g takes the
-// CTA's tiles g, g + 2, ... The producer of a group loads the slot of each of
-// its tiles into the group's S_hi tile and streams the tile's chunks (k, q,
-// gk and v rows, gate scalars) through the group's ring of vector stages.
+// CTA's tiles g, g + 2, ... The producer of a group streams each tile's
+// chunks (k, q, gk and v rows, gate scalars) through the group's ring of
+// vector stages, and loads the tile's slot into the group's S_hi tile right
+// after its first chunk (the group frees S_hi of its previous tile only once
+// it has that chunk).
 // Both sides derive the chunk schedule from the item's length and committed
 // count, read from global memory, so neither depends on data that may not
 // have landed.
@@ -89,6 +98,22 @@ __device__ __forceinline__ void pf_item(const DecodeParams& p, int b, int& L, in
   n = n < 0 ? 0 : (n > L ? L : n);
 }
 
+// One tile's coordinates: item b, value head h, column slice, the item's
+// slot s, valid tokens L, committed count n, and its output block.
+struct PfTile {
+  int b, h, slice, s, L, n;
+  uint16_t* out;
+};
+__device__ __forceinline__ PfTile pf_tile(const DecodeParams& p, int tile, int n_slices) {
+  PfTile t;
+  t.slice = tile % n_slices;
+  t.h = (tile / n_slices) % p.H_v;
+  t.b = tile / (n_slices * p.H_v);
+  pf_item(p, t.b, t.L, t.n, t.s);
+  t.out = p.out + (static_cast<size_t>(t.b) * p.H_v + t.h) * p.T * p.D_v + t.slice * kTcVS;
+  return t;
+}
+
 // End of the chunk that starts at `pos`: the next multiple of kPfChunk, L, or
 // the committed count n when it falls inside.
 __device__ __forceinline__ int pf_chunk_end(int pos, int L, int n) {
@@ -119,25 +144,14 @@ __device__ __forceinline__ void pf_state_from_tile(uint32_t s_lane, const uint8_
   tmem_wait_st();
 }
 
-// Row i of the tile in tensor memory scaled by c.
-__device__ __forceinline__ void pf_state_scale(uint32_t s_lane, float c) {
-#pragma unroll
-  for (int k = 0; k < kTcVS / 32; ++k) {
-    uint32_t r[32];
-    tmem_ld32(s_lane + 32 * k, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(c * __uint_as_float(r[e]));
-    tmem_st32(s_lane + 32 * k, r);
-  }
-  tmem_wait_st();
-}
-
 // Row i of the tile from tensor memory into the swizzled S_hi (bf16 RNE) and,
-// when LO, S_lo (the rounding remainder, bf16) tiles.
-template <bool LO>
+// when LO, S_lo (the rounding remainder, bf16) tiles; when SCALE, the row is
+// written back to tensor memory multiplied by c (the next chunk's decay).
+template <bool LO, bool SCALE>
 __device__ __forceinline__ void pf_state_to_tiles(uint32_t s_lane, uint8_t* s_hi, uint8_t* s_lo,
-                                                  int i) {
+                                                  int i, float c) {
+  const unsigned long long cc = pk(c, c);
+  const unsigned long long neg1 = pk(-1.0f, -1.0f);
 #pragma unroll
   for (int k = 0; k < kTcVS / 32; ++k) {
     uint32_t r[32];
@@ -145,16 +159,34 @@ __device__ __forceinline__ void pf_state_to_tiles(uint32_t s_lane, uint8_t* s_hi
     tmem_wait_ld();
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float x[8];
+      uint32_t hw[4], lw[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(r[8 * q + e]);
-      uint4 hi, lo;
-      split_bf16x8(x, hi, lo);
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(r[8 * q + 2 * e]);
+        const float x1 = __uint_as_float(r[8 * q + 2 * e + 1]);
+        hw[e] = pack_bf16x2(x0, x1);  // bf16 round to nearest even
+        if constexpr (LO) {
+          // the remainder x - bf16(x), exact in fp32, rounded to bf16
+          const float2 rem = upk(fma2(pk(bf16_lo(hw[e]), bf16_hi(hw[e])), neg1, pk(x0, x1)));
+          lw[e] = pack_bf16x2(rem.x, rem.y);
+        }
+      }
       const int off = swz_offset<kTcDK>(i, 32 * k + 8 * q);
-      *reinterpret_cast<uint4*>(s_hi + off) = hi;
-      if constexpr (LO) *reinterpret_cast<uint4*>(s_lo + off) = lo;
+      *reinterpret_cast<uint4*>(s_hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      if constexpr (LO)
+        *reinterpret_cast<uint4*>(s_lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    if constexpr (SCALE) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const float2 v = upk(mul2(cc, pk(__uint_as_float(r[e]), __uint_as_float(r[e + 1]))));
+        r[e] = __float_as_uint(v.x);
+        r[e + 1] = __float_as_uint(v.y);
+      }
+      tmem_st32(s_lane + 32 * k, r);
     }
   }
+  if constexpr (SCALE) tmem_wait_st();
 }
 
 // Row i of the S_lo tile cleared (the slot's bf16 state is exact in S_hi).
@@ -247,19 +279,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int b = tile / (n_slices * p.H_v);
       int L, n, s;
       pf_item(p, b, L, n, s);
-      if (L > 0) {  // the slot's state into S_hi, once S_hi is free
-        bool ok = true;
-        if (lane == 0)
-          ok = mbar_wait_abandonable(sempty, (fills & 1) ^ 1, abort_word, kErrProducerWait);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        if (lane == 0) {
-          mbar_expect_tx(sfull, kTcStateBytes);
-          tma_load_3d(smem_addr(s_hi), &pool_map, 0, (s * p.H_v + h) * DK, slice * VS / 64,
-                      sfull);
-          mbar_arrive(sfull);
-        }
-        ++fills;
-      }
       int pos = 0;
       do {  // one record per chunk; an empty item has one record of no tokens
         const int end = L > 0 ? pf_chunk_end(pos, L, n) : 0;
@@ -314,6 +333,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         cp_async_arrive_noinc(vbar);
         ++rec;
+        if (pos == 0 && L > 0) {
+          // the slot's state into S_hi once S_hi is free: after the tile's first
+          // record, which the group waits for before it frees S_hi of its
+          // previous tile
+          bool ok_s = true;
+          if (lane == 0)
+            ok_s = mbar_wait_abandonable(sempty, (fills & 1) ^ 1, abort_word, kErrProducerWait);
+          if (!__shfl_sync(0xffffffffu, ok_s, 0)) {
+            stop = true;
+            break;
+          }
+          if (lane == 0) {
+            mbar_expect_tx(sfull, kTcStateBytes);
+            tma_load_3d(smem_addr(s_hi), &pool_map, 0, (s * p.H_v + h) * DK, slice * VS / 64,
+                        sfull);
+            mbar_arrive(sfull);
+          }
+          ++fills;
+        }
         pos = end;
       } while (pos < L);
     }
@@ -349,150 +387,95 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     bool dead = false;  // a wait of the group failed (by vote): no commit, no signal
     bool storing = false;  // a TMA store may still be reading S_hi (elected thread)
 
-    for (int it = group; it < n_mine; it += kPfGroups) {
-      const int tile = blockIdx.x + it * gridDim.x;
-      const int slice = tile % n_slices;
-      const int h = (tile / n_slices) % p.H_v;
-      const int b = tile / (n_slices * p.H_v);
-      int L, n, s;
-      pf_item(p, b, L, n, s);
-      uint16_t* out_tile = p.out + (static_cast<size_t>(b) * p.H_v + h) * T * p.D_v + slice * VS;
-      const int fill = fills;
-      if (L > 0) ++fills;
-      int pos = 0;
-      do {
-        const int end = L > 0 ? pf_chunk_end(pos, L, n) : 0;
-        const int Lc = end - pos;
-        const bool first = pos == 0 && L > 0;
-        const bool last = end >= L;
-        const bool commit_here = n > 0 && end == n;
-        const int stage = rec % kPfStages;
-        const uint8_t* vb = vec_base + stage * vec_bytes;
-        bool ok_self = dead ? false
-                            : mbar_wait_abandonable(vfull0 + 8 * stage, (rec / kPfStages) & 1,
-                                                    abort_word, kErrConsumerWait);
-        int Lw = __all_sync(0xffffffffu, ok_self) ? Lc : 0;  // one value per warp
+    // Records are taken one behind: the iteration that prepares record k (waits
+    // for its rows, finalises them) first reads back the state that record
+    // k - 1 left in tensor memory into S_hi / S_lo, and, when k continues the
+    // same tile, writes it back to tensor memory already scaled by k's decay c.
+    // A tile's commit and wrap-up follow that read-back. One loop iteration
+    // per record plus one to finish the last; the finalise and solve code sit
+    // in the loop once.
+    int it = group;  // the tile of the record being prepared
+    int pos = 0;
+    PfTile cur{}, prev{};
+    if (it < n_mine) cur = pf_tile(p, blockIdx.x + it * gridDim.x, n_slices);
+    int fill = 0;
+    if (it < n_mine && cur.L > 0) ++fills;
+    bool have_prev = false, prev_last = false, prev_commit = false;
+    int prev_Lw = 0;
+    while (it < n_mine || have_prev) {
+      const bool has_cur = it < n_mine;
+      int end = 0;
+      bool first = false, last = false, commit_here = false;
+      if (has_cur) {
+        end = cur.L > 0 ? pf_chunk_end(pos, cur.L, cur.n) : 0;
+        first = pos == 0 && cur.L > 0;
+        last = end >= cur.L;
+        commit_here = cur.n > 0 && end == cur.n;
+      }
+      const int stage = rec % kPfStages;
+      const uint8_t* vb = vec_base + stage * vec_bytes;
 
-        // ---- finalise: row i = r (decays, u, w, e, c, partial sums of A and B)
-        float c_row = 0.0f, b_lane = 0.0f;
+      // ---- this record's rows: wait, then finalise row i = r (decays, u, w,
+      // e, c, partial sums of A and B)
+      bool ok_self = true;
+      int Lw = 0;
+      float c_row = 0.0f, b_lane = 0.0f;
+      if (has_cur) {
+        ok_self = dead ? false
+                       : mbar_wait_abandonable(vfull0 + 8 * stage, (rec / kPfStages) & 1,
+                                               abort_word, kErrConsumerWait);
+        Lw = __all_sync(0xffffffffu, ok_self) ? end - pos : 0;  // one value per warp
         if (Lw > 0) {
           float gt = 0.0f;
           if (lane < Lw) {
             const uint32_t* rawv = reinterpret_cast<const uint32_t*>(vb + lay.raw);
             if constexpr (GATED) {
-              const size_t ai = (static_cast<size_t>(b) * T + pos + lane) * p.H_v + h;
+              const size_t ai = (static_cast<size_t>(cur.b) * T + pos + lane) * p.H_v + cur.h;
               const float dtb = __uint_as_float(rawv[16]);
               const float dsc = __uint_as_float(rawv[17]);
               gt = dsc * softplus_f32(bf16_in_word(rawv[lane], p.gate_a + ai) + dtb);  // g
               b_lane = sigmoid_f32(bf16_in_word(rawv[8 + lane], p.gate_b + ai));      // beta
             } else {
-              const size_t gi = (static_cast<size_t>(b) * p.H_v + h) * T + pos + lane;
+              const size_t gi = (static_cast<size_t>(cur.b) * p.H_v + cur.h) * T + pos + lane;
               gt = __uint_as_float(rawv[lane]);
               b_lane = bf16_in_word(rawv[8 + lane], p.beta + gi);
             }
           }
-          c_row = tc_finalize_any<true>(Lw, Lw, vb, lay, gb, gt, p.scale, r, lane, wq);
+          c_row = tc_finalize<kPfChunk, true>(vb, lay, gb, gt, p.scale, r, lane, wq, Lw, Lw);
         }
-        if (first) {
-          ok_self = ok_self &&
-                    mbar_wait_abandonable(sfull, fill & 1, abort_word, kErrConsumerWait);
-          pf_zero_row(s_lo, r);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        // operands written; D1 free; the vote: the chunk goes on only if every
-        // thread saw its rows (and, first, the slot's state) land
-        if (!named_barrier_and(bar_id, kTcGroupThreads, ok_self)) {
-          dead = true;
-          Lw = 0;
-        }
+        if (first) pf_zero_row(s_lo, r);  // the slot's bf16 state is exact in S_hi
+      }
 
-        if (Lw > 0) {
-          // ---- pass 1: D1 = S_hi^T B1 + S_lo^T B1
-          if (wq == 0) {
-            if (elect_one()) {
-              tc_fence_after();
-#pragma unroll
-              for (int ks = 0; ks < DK / 16; ++ks)
-                umma_bf16(d1, umma_desc_advance(hi_desc, ks * 2048),
-                          umma_desc_advance(b1_desc, ks * 256), idesc1, ks > 0);
-#pragma unroll
-              for (int ks = 0; ks < DK / 16; ++ks)
-                umma_bf16(d1, umma_desc_advance(lo_desc, ks * 2048),
-                          umma_desc_advance(b1_desc, ks * 256), idesc1, true);
-              umma_commit(mbar);
-            }
-            __syncwarp();
-          }
-          // the state in TMEM scaled by c while pass 1 runs (it reads only the tiles)
-          tc_fence_after();
-          if (first)
-            pf_state_from_tile(s_tm + lane_field, s_hi, c_row, r);
-          else
-            pf_state_scale(s_tm + lane_field, c_row);
-          tc_sum_parts(gb, Lw, r);
-        }
-        tc_fence_before();
-        named_barrier(bar_id, kTcGroupThreads);  // A and B summed; the state scaled
+      // ---- the previous record's state back into the tiles (and, within a
+      // tile, into tensor memory scaled by this record's c)
+      if (have_prev && prev_Lw > 0) {
+        tc_fence_after();
+        if (!prev_last)
+          pf_state_to_tiles<true, true>(s_tm + lane_field, s_hi, s_lo, r, c_row);
+        else if (prev_commit)
+          pf_state_to_tiles<false, false>(s_tm + lane_field, s_hi, s_lo, r, 0.0f);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      // operands and state tiles written, TMEM reads done; the vote: this
+      // record goes on only if every thread saw its rows land
+      if (!named_barrier_and(bar_id, kTcGroupThreads, ok_self)) {
+        dead = true;
+        Lw = 0;
+      }
 
-        // ---- solve: column j = r; outputs of tokens pos .. end - 1
-        if (Lw > 0) {
-          if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
-          mma_phase ^= 1u;
-          tc_fence_after();
-          uint32_t x[32];
-          tmem_ld32(d1 + lane_field, x);
-          tmem_wait_ld();
-          tc_solve_any(Lw, x, vb, lay, gb, reinterpret_cast<const float*>(gb + kTcA),
-                       reinterpret_cast<const float*>(gb + kTcBm), b_lane, r,
-                       out_tile + static_cast<size_t>(pos) * p.D_v, p.D_v);
-        }
-        if (elected && storing && Lw > 0) {  // S_hi is rewritten below
-          bulk_wait_read_all();
-          storing = false;
-        }
-        fence_async_smem();
-        tc_fence_before();
-        named_barrier(bar_id, kTcGroupThreads);  // delta written; D1 and the stage read
-        if (elected && !dead) mbar_arrive(vempty0 + 8 * stage);
-
-        // ---- pass 2 into the state, then the state back into S_hi / S_lo
-        const bool stage_lo = !last;           // the next chunk's pass 1 reads S_lo
-        const bool need_tiles = !last || commit_here;
-        if (Lw > 0) {
-          if (wq == 0) {
-            if (elect_one()) {
-              tc_fence_after();
-#pragma unroll
-              for (int ks = 0; ks < kTcK2 / 16; ++ks)
-                umma_bf16(s_tm, umma_desc_advance(e_desc, ks * 256),
-                          umma_desc_advance(dl_desc, ks * 256), idesc2, true);
-              umma_commit(mbar);
-            }
-            __syncwarp();
-          }
-          if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
-          mma_phase ^= 1u;
-          tc_fence_after();
-          if (need_tiles) {
-            if (stage_lo)
-              pf_state_to_tiles<true>(s_tm + lane_field, s_hi, s_lo, r);
-            else
-              pf_state_to_tiles<false>(s_tm + lane_field, s_hi, s_lo, r);
-          }
-          fence_async_smem();
-        }
-        tc_fence_before();
-        named_barrier(bar_id, kTcGroupThreads);  // new state staged; TMEM reads done
-        if (elected && Lw > 0 && commit_here) {
-          tma_store_3d(&pool_map, 0, (s * p.H_v + h) * DK, slice * VS / 64, smem_addr(s_hi));
+      // ---- the previous record's commit, and the wrap-up of its tile
+      if (have_prev) {
+        if (elected && prev_Lw > 0 && prev_commit) {
+          tma_store_3d(&pool_map, 0, (prev.s * p.H_v + prev.h) * DK, prev.slice * VS / 64,
+                       smem_addr(s_hi));
           bulk_commit_group();
           storing = true;
         }
-        if (last) {
+        if (prev_last) {
           // padded tokens (and every token of an empty or skipped item): +0.0
-          pf_zero_out(out_tile, L, T, p.D_v, r);
-          if (L > 0 && elected) {  // S_hi is free once the store has read it
+          pf_zero_out(prev.out, prev.L, T, p.D_v, r);
+          if (prev.L > 0 && elected) {  // S_hi is free once the store has read it
             if (storing) {
               bulk_wait_read_all();
               storing = false;
@@ -500,9 +483,99 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (!dead) mbar_arrive(sempty);
           }
         }
-        ++rec;
-        pos = end;
-      } while (pos < L);
+      }
+      if (!has_cur) break;
+      if (first) {  // the slot's state landed in S_hi, by vote
+        const bool ok_state =
+            !dead && mbar_wait_abandonable(sfull, fill & 1, abort_word, kErrConsumerWait);
+        if (!named_barrier_and(bar_id, kTcGroupThreads, ok_state)) {
+          dead = true;
+          Lw = 0;
+        }
+      }
+
+      if (Lw > 0) {
+        // ---- pass 1: D1 = S_hi^T B1 + S_lo^T B1
+        if (wq == 0) {
+          if (elect_one()) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < DK / 16; ++ks)
+              umma_bf16(d1, umma_desc_advance(hi_desc, ks * 2048),
+                        umma_desc_advance(b1_desc, ks * 256), idesc1, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < DK / 16; ++ks)
+              umma_bf16(d1, umma_desc_advance(lo_desc, ks * 2048),
+                        umma_desc_advance(b1_desc, ks * 256), idesc1, true);
+            umma_commit(mbar);
+          }
+          __syncwarp();
+        }
+        // a tile's first record: the state into TMEM as c S_0 while pass 1 runs
+        // (it reads only the tiles); later records find it scaled already
+        if (first) {
+          tc_fence_after();
+          pf_state_from_tile(s_tm + lane_field, s_hi, c_row, r);
+        }
+        tc_sum_parts(gb, Lw, r);
+      }
+      tc_fence_before();
+      named_barrier(bar_id, kTcGroupThreads);  // A and B summed; the state in TMEM
+
+      // ---- solve: column j = r; outputs of tokens pos .. end - 1
+      if (Lw > 0) {
+        if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
+        mma_phase ^= 1u;
+        tc_fence_after();
+        uint32_t x[32];
+        tmem_ld32(d1 + lane_field, x);
+        tmem_wait_ld();
+        tc_solve<kPfChunk>(x, vb, lay, gb, reinterpret_cast<const float*>(gb + kTcA),
+                           reinterpret_cast<const float*>(gb + kTcBm), b_lane, r,
+                           cur.out + static_cast<size_t>(pos) * p.D_v, p.D_v, Lw);
+      }
+      if (elected && storing && Lw > 0) {  // S_hi is rewritten by the next read-back
+        bulk_wait_read_all();
+        storing = false;
+      }
+      fence_async_smem();
+      tc_fence_before();
+      named_barrier(bar_id, kTcGroupThreads);  // delta written; D1 and the stage read
+      if (elected && !dead) mbar_arrive(vempty0 + 8 * stage);
+
+      // ---- pass 2 into the state
+      if (Lw > 0) {
+        if (wq == 0) {
+          if (elect_one()) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < kTcK2 / 16; ++ks)
+              umma_bf16(s_tm, umma_desc_advance(e_desc, ks * 256),
+                        umma_desc_advance(dl_desc, ks * 256), idesc2, true);
+            umma_commit(mbar);
+          }
+          __syncwarp();
+        }
+        if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
+        mma_phase ^= 1u;
+      }
+
+      have_prev = true;
+      prev_Lw = Lw;
+      prev_last = last;
+      prev_commit = commit_here;
+      prev = cur;
+      ++rec;
+      pos = end;
+      if (pos >= cur.L) {  // the tile's last record: on to the group's next tile
+        it += kPfGroups;
+        pos = 0;
+        if (it < n_mine) {
+          cur = pf_tile(p, blockIdx.x + it * gridDim.x, n_slices);
+          fill = fills;
+          if (cur.L > 0) ++fills;
+        }
+      }
     }
     if (elected) bulk_wait_all();
   }

@@ -46,6 +46,8 @@ def hooks():
     L = ctypes.CDLL(path)
     L.gdr_decode.argtypes = binding._DECODE_ARGTYPES
     L.gdr_decode.restype = ctypes.c_int
+    L.gdr_prefill.argtypes = binding._DECODE_ARGTYPES
+    L.gdr_prefill.restype = ctypes.c_int
     L.gdr_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
     L.gdr_device_error.restype = ctypes.c_int
     L.gdr_last_launch.argtypes = [ctypes.POINTER(binding.LaunchInfo)]
@@ -57,18 +59,20 @@ def hooks():
     assert L.gdrtest_set_hooks(0, -1) == 0
 
 
-def _decode(L, xd, state_layout="kv"):
-    """gdr_decode of the test build, with the binding's argument checks."""
+def _decode(L, xd, state_layout="kv", prefill=False):
+    """gdr_decode (or gdr_prefill) of the test build, with the binding's
+    argument checks."""
     from gated_delta_rule_recurrent_b200 import binding
 
     _, dims, out, stream = binding._common(
         xd["query"], xd["key"], xd["value"], xd["state_pool"], xd["actual_seq_lengths"],
         xd["ssm_state_indices"], xd["gk"], xd["num_accepted_tokens"], None, state_layout)
     P = binding._ptr
-    rc = L.gdr_decode(ctypes.byref(dims), P(xd["query"]), P(xd["key"]), P(xd["value"]),
-                      P(xd["beta"]), P(xd["state_pool"]), P(xd["actual_seq_lengths"]),
-                      P(xd["ssm_state_indices"]), P(xd["g"]), P(xd["gk"]),
-                      P(xd["num_accepted_tokens"]), float(xd["scale_value"]), P(out), stream)
+    entry = L.gdr_prefill if prefill else L.gdr_decode
+    rc = entry(ctypes.byref(dims), P(xd["query"]), P(xd["key"]), P(xd["value"]),
+               P(xd["beta"]), P(xd["state_pool"]), P(xd["actual_seq_lengths"]),
+               P(xd["ssm_state_indices"]), P(xd["g"]), P(xd["gk"]),
+               P(xd["num_accepted_tokens"]), float(xd["scale_value"]), P(out), stream)
     assert rc == 0, L.gdr_last_error().decode()
     return out
 
@@ -88,18 +92,22 @@ def _grid(L):
 
 
 # (what, D_k, D_v, H, B, T): one shape per kernel family, with more tiles than
-# SMs so that CTA 0 has a tile before the held one
+# SMs so that CTA 0 has a tile before the held one. In the prefill kernel the
+# held tile is the first one of CTA 0's second consumer group, whose first
+# group keeps working beside it.
 FAMILIES = [
     ("single_token", 64, 512, 4, 40, 1),
     ("chunked", 64, 512, 4, 6, 3),
     ("tensor_core", 128, 128, 4, 40, 3),
     ("tensor_core_one", 128, 128, 4, 40, 1),
+    ("prefill", 128, 128, 4, 40, 20),
 ]
 
 
 @pytest.mark.parametrize("what,D_k,D_v,H,B,T", FAMILIES, ids=[f[0] for f in FAMILIES])
 def test_held_tile_times_out_cleanly(hooks, what, D_k, D_v, H, B, T):
     L = hooks
+    pf = what == "prefill"
     w = workloads.WORKLOADS[0].replace(name=f"hold_{what}", B=B, H_qk=H, H_v=H, T=T, D_k=D_k,
                                        D_v=D_v, pool=B + 2, lengths="full", indices="subset",
                                        scale_value=D_k**-0.5, seed=77 + D_k + T)
@@ -110,7 +118,7 @@ def test_held_tile_times_out_cleanly(hooks, what, D_k, D_v, H, B, T):
     assert L.gdrtest_set_hooks(0, -1) == 0
     _error_word(L)
     xd = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    _decode(L, xd)
+    _decode(L, xd, prefill=pf)
     torch.cuda.synchronize()
     launch = _grid(L)
     assert launch["kernel"] == what, launch
@@ -125,7 +133,7 @@ def test_held_tile_times_out_cleanly(hooks, what, D_k, D_v, H, B, T):
     xd = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     assert L.gdrtest_set_hooks(SHORT_BUDGET, held) == 0
     t0 = time.perf_counter()
-    _decode(L, xd)
+    _decode(L, xd, prefill=pf)
     torch.cuda.synchronize()
     elapsed = time.perf_counter() - t0
     assert L.gdrtest_set_hooks(0, -1) == 0
@@ -157,7 +165,7 @@ def test_held_tile_times_out_cleanly(hooks, what, D_k, D_v, H, B, T):
 
     # the device is healthy: a normal call right after passes parity
     xd = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
-    out = _decode(L, xd)
+    out = _decode(L, xd, prefill=pf)
     torch.cuda.synchronize()
     check_call(x, out, pool0, xd["state_pool"].cpu(), False)
     assert _error_word(L) == 0
