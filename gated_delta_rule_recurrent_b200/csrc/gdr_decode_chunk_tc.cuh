@@ -804,7 +804,15 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
             b_lane = bf16_in_word(rawv[8 + lane], p.beta + gi);
           }
         }
-        c_row = tc_finalize_any<!SUMS>(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
+        // T = 8: two instances cover every length (L <= 4 and L <= 8; the
+        // stage holds 8 rows and the tokens past L are masked), so a mix of
+        // lengths runs two copies of the code instead of eight
+        if (!SUMS && T == 8 && L <= 4)
+          c_row = tc_finalize<4, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
+        else if (!SUMS && T == 8)
+          c_row = tc_finalize<8, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
+        else
+          c_row = tc_finalize_any<!SUMS>(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
         if constexpr (VK) reinterpret_cast<float*>(gb + kTcC)[r] = c_row;
       }
       fence_async_smem();
@@ -868,7 +876,14 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         const float* sa = SUMS ? reinterpret_cast<const float*>(vb + lay.ab)
                                : reinterpret_cast<const float*>(gb + kTcA);
         const float* sb = SUMS ? sa + 64 : reinterpret_cast<const float*>(gb + kTcBm);
-        if (sums_ok) tc_solve_any(L, x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
+        if (sums_ok) {
+          if (!SUMS && T == 8 && L <= 4)
+            tc_solve<4>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
+          else if (!SUMS && T == 8)
+            tc_solve<8>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
+          else
+            tc_solve_any(L, x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
+        }
       }
       fence_async_smem();
       tc_fence_before();
