@@ -331,7 +331,7 @@ int launch_chunk(const gdr::DecodeParams& p, cudaStream_t stream) {
 
 // One persistent CTA per SM with kTcGroups consumer groups; each group gets
 // as many stages as shared memory holds (at most 4).
-template <bool GATED, bool VK, bool SUMS>
+template <bool GATED, bool VK, bool SUMS, bool T8>
 int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) {
   static ChunkConfig cache[kMaxDevices][gdr::kMaxT + 1];
   static std::atomic<bool> ready[kMaxDevices][gdr::kMaxT + 1];
@@ -339,7 +339,7 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
     *out = cache[dev][T];
     return GDR_OK;
   }
-  auto kernel = gdr::decode_chunk_tc_kernel<GATED, VK, SUMS>;
+  auto kernel = gdr::decode_chunk_tc_kernel<GATED, VK, SUMS, T8>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          props.smem_optin);
   if (err == cudaSuccess)
@@ -367,7 +367,7 @@ int chunk_tc_config(int dev, int T, const DeviceProps& props, ChunkConfig* out) 
   return GDR_OK;
 }
 
-template <bool GATED, bool VK, bool SUMS>
+template <bool GATED, bool VK, bool SUMS, bool T8>
 int launch_chunk_tc_sums(const gdr::DecodeParams& p, cudaStream_t stream) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
@@ -376,14 +376,14 @@ int launch_chunk_tc_sums(const gdr::DecodeParams& p, cudaStream_t stream) {
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   ChunkConfig cfg;
-  rc = chunk_tc_config<GATED, VK, SUMS>(dev, p.T, props, &cfg);
+  rc = chunk_tc_config<GATED, VK, SUMS, T8>(dev, p.T, props, &cfg);
   if (rc != GDR_OK) return rc;
   CUtensorMap map;
   rc = encode_pool_map(p, gdr::kTcDK, gdr::kTcVS, VK, &map);
   if (rc != GDR_OK) return rc;
   const int n_tiles = p.B * p.H_v * (p.D_v / gdr::kTcVS);
   const int grid = n_tiles < props.sms ? n_tiles : props.sms;
-  gdr::decode_chunk_tc_kernel<GATED, VK, SUMS><<<grid, cfg.threads, cfg.smem, stream>>>(
+  gdr::decode_chunk_tc_kernel<GATED, VK, SUMS, T8><<<grid, cfg.threads, cfg.smem, stream>>>(
       map, p, n_tiles, cfg.n_stages);
   err = cudaGetLastError();
   if (err != cudaSuccess)
@@ -396,8 +396,9 @@ int launch_chunk_tc_sums(const gdr::DecodeParams& p, cudaStream_t stream) {
 // Single-token calls take the sums-warp form of the kernel.
 template <bool GATED, bool VK>
 int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
-  return p.T == 1 ? launch_chunk_tc_sums<GATED, VK, true>(p, stream)
-                  : launch_chunk_tc_sums<GATED, VK, false>(p, stream);
+  return p.T == 1   ? launch_chunk_tc_sums<GATED, VK, true, false>(p, stream)
+         : p.T == 8 ? launch_chunk_tc_sums<GATED, VK, false, true>(p, stream)
+                    : launch_chunk_tc_sums<GATED, VK, false, false>(p, stream);
 }
 
 using LaunchFn = int (*)(const gdr::DecodeParams&, cudaStream_t);

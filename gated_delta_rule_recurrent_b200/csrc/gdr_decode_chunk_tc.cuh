@@ -439,7 +439,8 @@ __device__ __forceinline__ void tc_solve_any(int L, const uint32_t (&x)[32], con
 // chunks read from shared memory while they are.
 __device__ __forceinline__ void tc_new_state_row(uint8_t* st, uint32_t d2_lane, float c, int i) {
   const unsigned long long cc = pk(c, c);
-#pragma unroll
+#pragma unroll 1  // two rounds as a loop: half the code, measured faster
+
   for (int k = 0; k < kTcVS / 64; ++k) {
     uint32_t acc[2][32];
     tmem_ld32(d2_lane + 64 * k, acc[0]);
@@ -481,7 +482,9 @@ __device__ __forceinline__ void tc_new_state_row(uint8_t* st, uint32_t d2_lane, 
 // stages (n_stages a multiple of n_groups) and takes them in turn, so a stage
 // passes only between the producer and one group, which has waited for the
 // stage's previous fill before it waits for the next: no wait can see a phase
-// two fills old.
+// two fills old. T8 marks the instance that T = 8 calls launch (the row and
+// column code for L <= 4 and L <= 8 only); other multi-token calls take the
+// instance with all eight token counts.
 __device__ __forceinline__ int tc_stage(int j, int n_groups, int per_group) {
   return (j % n_groups) * per_group + (j / n_groups) % per_group;
 }
@@ -493,7 +496,7 @@ __device__ __forceinline__ uint32_t tc_phase(int j, int n_groups, int per_group)
 // over the staged tile [D_k / 64][VS rows j][64] (c from shared memory).
 __device__ __forceinline__ void tc_new_state_row_vk(uint8_t* st, uint32_t d2_lane, const float* c,
                                                     int j) {
-#pragma unroll
+#pragma unroll 1  // as tc_new_state_row
   for (int k = 0; k < kTcDK / 64; ++k) {
     uint32_t acc[2][32];
     tmem_ld32(d2_lane + 64 * k, acc[0]);
@@ -525,7 +528,7 @@ __device__ __forceinline__ void tc_new_state_row_vk(uint8_t* st, uint32_t d2_lan
   }
 }
 
-template <bool GATED, bool VK, bool SUMS>
+template <bool GATED, bool VK, bool SUMS, bool T8>
 __global__ void __launch_bounds__(kTcMaxThreads, 1)
     decode_chunk_tc_kernel(const __grid_constant__ CUtensorMap pool_map, const DecodeParams p,
                            const int n_tiles, const int n_stages) {
@@ -728,8 +731,8 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
             gt = __uint_as_float(rawv[lane]);
           }
         }
-        tc_pair_sums_any(L, vb, lay, reinterpret_cast<float*>(const_cast<uint8_t*>(vb) + lay.ab),
-                         gt, p.scale, lane);
+        tc_pair_sums<1>(vb, lay, reinterpret_cast<float*>(const_cast<uint8_t*>(vb) + lay.ab), gt,
+                        p.scale, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(ab0 + 8 * stage);
@@ -804,15 +807,21 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
             b_lane = bf16_in_word(rawv[8 + lane], p.beta + gi);
           }
         }
-        // T = 8: two instances cover every length (L <= 4 and L <= 8; the
-        // stage holds 8 rows and the tokens past L are masked), so a mix of
-        // lengths runs two copies of the code instead of eight
-        if (!SUMS && T == 8 && L <= 4)
-          c_row = tc_finalize<4, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
-        else if (!SUMS && T == 8)
-          c_row = tc_finalize<8, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
-        else
+        // The code a call runs is kept small (instruction fetch is a leading
+        // stall here): T = 8 kernels hold two instances that cover every
+        // length (L <= 4 and L <= 8; the stage holds 8 rows and the tokens
+        // past L are masked), single-token kernels the L = 1 one, and only
+        // the other token counts take the switch over all eight.
+        if constexpr (T8) {
+          if (L <= 4)
+            c_row = tc_finalize<4, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
+          else
+            c_row = tc_finalize<8, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
+        } else if constexpr (SUMS) {  // single-token calls: L = 1
+          c_row = tc_finalize<1, false>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit);
+        } else {
           c_row = tc_finalize_any<!SUMS>(L, n_commit, vb, lay, gb, gt, p.scale, r, lane, wq);
+        }
         if constexpr (VK) reinterpret_cast<float*>(gb + kTcC)[r] = c_row;
       }
       fence_async_smem();
@@ -877,12 +886,16 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
                                : reinterpret_cast<const float*>(gb + kTcA);
         const float* sb = SUMS ? sa + 64 : reinterpret_cast<const float*>(gb + kTcBm);
         if (sums_ok) {
-          if (!SUMS && T == 8 && L <= 4)
-            tc_solve<4>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
-          else if (!SUMS && T == 8)
-            tc_solve<8>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
-          else
+          if constexpr (T8) {
+            if (L <= 4)
+              tc_solve<4>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
+            else
+              tc_solve<8>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
+          } else if constexpr (SUMS) {
+            tc_solve<1>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
+          } else {
             tc_solve_any(L, x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
+          }
         }
       }
       fence_async_smem();

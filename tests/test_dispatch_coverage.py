@@ -33,14 +33,18 @@ MIN_TILES_PER_SM = 16
 GUARD = 4096
 PATTERN = 0xA5
 
-# (kernel, D_k, tile_cols, layout, T, D_v, H): one call shape per kernel form;
-# each runs with and without the fused gate. B is derived at run time.
+# (kernel, D_k, tile_cols, layout, T, D_v, H): one call shape per kernel form,
+# and one more where a form has a separate instance for some token count (the
+# tensor-core kernel at T = 8); each runs with and without the fused gate. B
+# is derived at run time.
 CASES = [
     ("prefill", 128, 128, "kv", 21, 256, 4),
     ("tensor_core_one", 128, 128, "kv", 1, 256, 4),
     ("tensor_core", 128, 128, "kv", 5, 256, 4),
+    ("tensor_core", 128, 128, "kv", 8, 256, 4),  # the instance built for T = 8
     ("tensor_core_one", 128, 128, "vk", 1, 256, 4),
     ("tensor_core", 128, 128, "vk", 5, 256, 4),
+    ("tensor_core", 128, 128, "vk", 8, 256, 4),
     ("single_token", 64, 512, "kv", 1, 512, 64),
     ("single_token", 64, 256, "kv", 1, 512, 64),
     ("single_token", 64, 128, "kv", 1, 512, 64),
