@@ -162,10 +162,15 @@ __device__ __forceinline__ void split_bf16x8(const float (&x)[8], uint4& hi, uin
 // in lane t. Returns c_i = P_{n-1}[i] (0 when n = 0). With nv < LC only the
 // first nv tokens are valid (n <= nv): u and w are zero past them, and the
 // sums that involve a later token are left unspecified (never read).
-template <int LC, bool PAIRS>
+// before_e() runs right before the e operand is written (a caller whose
+// previous pass 2 may still be reading it waits there).
+struct TcNoHook {
+  __device__ __forceinline__ void operator()() const {}
+};
+template <int LC, bool PAIRS, class BeforeE = TcNoHook>
 __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& lay, uint8_t* gb,
                                              float g_lane, float scale, int i, int lane, int wq,
-                                             int n, int nv = LC) {
+                                             int n, int nv = LC, BeforeE before_e = BeforeE()) {
   constexpr int DK = kTcDK;
   constexpr int NM = pow2_at_least(LC * LC);  // partial sums, padded for the reduce-scatter
   float g[LC];
@@ -221,6 +226,7 @@ __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& 
       }
     }
     split_bf16x8(e, hi, lo);
+    before_e();
     uint8_t* ep = gb + kTcE + (i >> 3) * 512 + (i & 7) * 16;
     *reinterpret_cast<uint4*>(ep) = hi;
     *reinterpret_cast<uint4*>(ep + 128) = hi;
@@ -251,6 +257,7 @@ __device__ __forceinline__ float tc_finalize(const uint8_t* vb, const TcLayout& 
     e[s] = es;
   }
   split_bf16x8(e, hi, lo);
+  before_e();
   uint8_t* ep = gb + kTcE + (i >> 3) * 512 + (i & 7) * 16;
   *reinterpret_cast<uint4*>(ep) = hi;
   *reinterpret_cast<uint4*>(ep + 128) = hi;

@@ -402,6 +402,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (it < n_mine && cur.L > 0) ++fills;
     bool have_prev = false, prev_last = false, prev_commit = false;
     int prev_Lw = 0;
+    // Pass 2 of the previous record is issued without a wait: this thread
+    // waits for it before the next finalise writes the e operand that pass 2
+    // reads (or, with no finalise, before the state is read back), so the
+    // MMA runs under the finalise's first part.
+    bool pending = false;
+    auto wait_pass2 = [&]() {
+      if (pending) {
+        if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
+        mma_phase ^= 1u;
+        pending = false;
+      }
+    };
     while (it < n_mine || have_prev) {
       const bool has_cur = it < n_mine;
       int end = 0;
@@ -441,13 +453,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               b_lane = bf16_in_word(rawv[8 + lane], p.beta + gi);
             }
           }
-          c_row = tc_finalize<kPfChunk, true>(vb, lay, gb, gt, p.scale, r, lane, wq, Lw, Lw);
+          c_row = tc_finalize<kPfChunk, true>(vb, lay, gb, gt, p.scale, r, lane, wq, Lw, Lw,
+                                              wait_pass2);
         }
         if (first) pf_zero_row(s_lo, r);  // the slot's bf16 state is exact in S_hi
       }
 
       // ---- the previous record's state back into the tiles (and, within a
       // tile, into tensor memory scaled by this record's c)
+      wait_pass2();
       if (have_prev && prev_Lw > 0) {
         tc_fence_after();
         if (!prev_last)
@@ -556,8 +570,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           __syncwarp();
         }
-        if (!mbar_wait_bounded(mbar, mma_phase)) flag_error(kErrConsumerWait);
-        mma_phase ^= 1u;
+        pending = true;
       }
 
       have_prev = true;
