@@ -815,10 +815,11 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
           }
         }
         // The code a call runs is kept small (instruction fetch is a leading
-        // stall here): T = 8 kernels hold two instances that cover every
-        // length (L <= 4 and L <= 8; the stage holds 8 rows and the tokens
-        // past L are masked), single-token kernels the L = 1 one, and only
-        // the other token counts take the switch over all eight.
+        // stall here): T = 8 kernels hold two finalise instances that cover
+        // every length (L <= 4 and L <= 8; the stage holds 8 rows and the
+        // tokens past L are masked) and one L <= 8 solve, single-token
+        // kernels the L = 1 code, and only the other token counts take the
+        // switch over all eight.
         if constexpr (T8) {
           if (L <= 4)
             c_row = tc_finalize<4, true>(vb, lay, gb, gt, p.scale, r, lane, wq, n_commit, L);
@@ -894,10 +895,7 @@ __global__ void __launch_bounds__(kTcMaxThreads, 1)
         const float* sb = SUMS ? sa + 64 : reinterpret_cast<const float*>(gb + kTcBm);
         if (sums_ok) {
           if constexpr (T8) {
-            if (L <= 4)
-              tc_solve<4>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
-            else
-              tc_solve<8>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
+            tc_solve<8>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v, L);
           } else if constexpr (SUMS) {
             tc_solve<1>(x, vb, lay, gb, sa, sb, b_lane, r, out_t0, p.D_v);
           } else {
