@@ -97,6 +97,27 @@ def test_empty_skipped_and_clamped_items(gated):
         assert np.all(ob[bi] == 0)
 
 
+@pytest.mark.parametrize("gated", [False, True])
+def test_long_prompt_past_the_bench_length(gated):
+    """T = 4096 (512 chunks per tile), one full-length item beside a ragged
+    one, two value heads sharing a q/k head."""
+    x = _prompt(4096, B=2, H_qk=1, H_v=2, seed=10, lengths="full")
+    x["actual_seq_lengths"] = torch.tensor([4096, 2999], dtype=torch.int32)
+    x["num_accepted_tokens"] = x["actual_seq_lengths"].clone()
+    _roundtrip(x, gated)
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_long_prompt_committed_mid_prompt(gated):
+    """n far inside a long prompt: the slot gets the state after n tokens
+    while outputs run on to L (reading E), with n on and off a chunk
+    boundary."""
+    x = _prompt(1000, B=3, seed=11, lengths="full")
+    x["actual_seq_lengths"] = torch.tensor([1000, 977, 640], dtype=torch.int32)
+    x["num_accepted_tokens"] = torch.tensor([500, 333, 640], dtype=torch.int32)
+    _roundtrip(x, gated)
+
+
 def test_one_token_prompt():
     _roundtrip(_prompt(1, B=4, seed=4, lengths="full"), False)
 
