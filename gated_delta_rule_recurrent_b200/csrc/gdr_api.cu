@@ -606,6 +606,16 @@ int launch_prefill(const gdr::DecodeParams& p, cudaStream_t stream) {
 
 // ---------------------------------------------------------------- standalone gate
 
+// CTAs of 256 threads a kernel keeps resident per SM (its registers decide),
+// queried once; the grid-stride grids are that many per SM, one wave.
+template <typename K>
+int resident_per_sm(K kernel) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1)
+    n = 1;
+  return n;
+}
+
 template <int TYPE, bool BETA>
 int launch_gate(const void* a, const void* b, const float* dt_bias, const float* decay_scale,
                 void* decay, void* beta, int64_t n, int H, cudaStream_t stream) {
@@ -617,28 +627,41 @@ int launch_gate(const void* a, const void* b, const float* dt_bias, const float*
   int rc = device_props(dev, &props);
   if (rc != GDR_OK) return rc;
   constexpr int kThreads = 256;
-  const int64_t max_blocks = static_cast<int64_t>(props.sms) * 8;  // 2048 threads per SM
-  auto blocks_for = [&](int64_t work) {
+  static const int res_head = resident_per_sm(gdr::gate_vec_kernel<TYPE, BETA, true>);
+  static const int res_elem = resident_per_sm(gdr::gate_vec_kernel<TYPE, BETA, false>);
+  static const int res_scalar = resident_per_sm(gdr::gate_scalar_kernel<TYPE, BETA>);
+  auto blocks_for = [&](int64_t work, int resident) {
+    const int64_t max_blocks = static_cast<int64_t>(props.sms) * resident;
     const int64_t blk = (work + kThreads - 1) / kThreads;
     return static_cast<int>(blk < max_blocks ? blk : max_blocks);
   };
   // 16-byte vectors when every tensor allows them; the rest element by element
   const bool vec = aligned16(a) && aligned16(decay) && (!BETA || (aligned16(b) && aligned16(beta)));
   const int64_t n_vec = vec ? n / E::kPerVec : 0;
-  if (n_vec > 0)
-    gdr::gate_vec_kernel<TYPE, BETA><<<blocks_for(n_vec), kThreads, 0, stream>>>(
-        static_cast<const uint4*>(a), static_cast<const uint4*>(b), dt_bias, decay_scale,
-        static_cast<uint4*>(decay), static_cast<uint4*>(beta), n_vec, H);
+  // per-head vectors as 16-byte loads when a vector's elements are whole heads
+  const bool headvec = H % E::kPerVec == 0 && aligned16(dt_bias) && aligned16(decay_scale);
+  const int vec_blocks = blocks_for(n_vec, headvec ? res_head : res_elem);
+  if (n_vec > 0) {
+    if (headvec)
+      gdr::gate_vec_kernel<TYPE, BETA, true><<<vec_blocks, kThreads, 0, stream>>>(
+          static_cast<const uint4*>(a), static_cast<const uint4*>(b), dt_bias, decay_scale,
+          static_cast<uint4*>(decay), static_cast<uint4*>(beta), n_vec, H);
+    else
+      gdr::gate_vec_kernel<TYPE, BETA, false><<<vec_blocks, kThreads, 0, stream>>>(
+          static_cast<const uint4*>(a), static_cast<const uint4*>(b), dt_bias, decay_scale,
+          static_cast<uint4*>(decay), static_cast<uint4*>(beta), n_vec, H);
+  }
   const int64_t i_begin = n_vec * E::kPerVec;
+  const int scalar_blocks = blocks_for(n - i_begin, res_scalar);
   if (i_begin < n)
-    gdr::gate_scalar_kernel<TYPE, BETA><<<blocks_for(n - i_begin), kThreads, 0, stream>>>(
+    gdr::gate_scalar_kernel<TYPE, BETA><<<scalar_blocks, kThreads, 0, stream>>>(
         static_cast<const bits*>(a), static_cast<const bits*>(b), dt_bias, decay_scale,
         static_cast<bits*>(decay), static_cast<bits*>(beta), i_begin, n, H);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess)
     return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
-  record_launch(GDR_KERNEL_GATE, 0, 0, true, false,
-                n_vec > 0 ? blocks_for(n_vec) : blocks_for(n - i_begin), kThreads, 0, 0);
+  record_launch(GDR_KERNEL_GATE, 0, 0, true, false, n_vec > 0 ? vec_blocks : scalar_blocks,
+                kThreads, 0, 0);
   return GDR_OK;
 }
 

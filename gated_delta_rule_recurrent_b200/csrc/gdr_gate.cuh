@@ -94,8 +94,12 @@ __device__ __forceinline__ void gate_elements(const typename GateElem<TYPE>::bit
 }
 
 // Vector path: n / kPerVec whole 16-byte vectors, all four tensors 16-byte
-// aligned; the scalar remainder is done by the caller's tail launch.
-template <int TYPE, bool BETA>
+// aligned; the scalar remainder is done by the caller's tail launch. When
+// HEADVEC (H a multiple of kPerVec and both per-head vectors 16-byte aligned),
+// a vector's kPerVec elements are heads h0 .. h0 + kPerVec - 1 and their
+// dt_bias and decay_scale come in as 16-byte loads. Each thread loads its next
+// vector's a (and b) before it works on the current one.
+template <int TYPE, bool BETA, bool HEADVEC>
 __global__ void __launch_bounds__(256) gate_vec_kernel(const uint4* __restrict__ a,
                                                        const uint4* __restrict__ b,
                                                        const float* __restrict__ dt_bias,
@@ -111,22 +115,45 @@ __global__ void __launch_bounds__(256) gate_vec_kernel(const uint4* __restrict__
   // head of this thread's first element, and how far it moves per stride
   int h0 = static_cast<int>((v * V) % H);
   const int h_step = static_cast<int>((stride * V) % H);
+  uint4 av_next = make_uint4(0u, 0u, 0u, 0u), bv_next = av_next;
+  if (v < n_vec) {
+    av_next = __ldcs(a + v);
+    if constexpr (BETA) bv_next = __ldcs(b + v);
+  }
   for (; v < n_vec; v += stride, h0 = h0 + h_step >= H ? h0 + h_step - H : h0 + h_step) {
-    const uint4 av = __ldcs(a + v);
-    uint4 bv;
-    if constexpr (BETA) bv = __ldcs(b + v);
+    const uint4 av = av_next;
+    const uint4 bv = bv_next;
+    if (v + stride < n_vec) {
+      av_next = __ldcs(a + v + stride);
+      if constexpr (BETA) bv_next = __ldcs(b + v + stride);
+    }
+    float dtb[V], dsc[V];
+    if constexpr (HEADVEC) {
+#pragma unroll
+      for (int q = 0; q < V / 4; ++q) {
+        const float4 t = __ldg(reinterpret_cast<const float4*>(dt_bias + h0) + q);
+        const float4 u = __ldg(reinterpret_cast<const float4*>(decay_scale + h0) + q);
+        dtb[4 * q] = t.x; dtb[4 * q + 1] = t.y; dtb[4 * q + 2] = t.z; dtb[4 * q + 3] = t.w;
+        dsc[4 * q] = u.x; dsc[4 * q + 1] = u.y; dsc[4 * q + 2] = u.z; dsc[4 * q + 3] = u.w;
+      }
+    } else {
+      int h = h0;
+#pragma unroll
+      for (int e = 0; e < V; ++e) {
+        dtb[e] = __ldg(dt_bias + h);
+        dsc[e] = __ldg(decay_scale + h);
+        h = h + 1 == H ? 0 : h + 1;
+      }
+    }
     const bits* ae = reinterpret_cast<const bits*>(&av);
     const bits* be = reinterpret_cast<const bits*>(&bv);
     uint4 dv, btv;
     bits* de = reinterpret_cast<bits*>(&dv);
     bits* bte = reinterpret_cast<bits*>(&btv);
-    int h = h0;
 #pragma unroll
     for (int e = 0; e < V; ++e) {
-      const float x = E::load(ae[e]) + __ldg(dt_bias + h);
-      de[e] = E::store(__ldg(decay_scale + h) * gate_softplus<E::kFast>(x));
+      de[e] = E::store(dsc[e] * gate_softplus<E::kFast>(E::load(ae[e]) + dtb[e]));
       if constexpr (BETA) bte[e] = E::store(gate_sigmoid<E::kFast>(E::load(be[e])));
-      h = h + 1 == H ? 0 : h + 1;
     }
     __stcs(decay + v, dv);
     if constexpr (BETA) __stcs(beta + v, btv);

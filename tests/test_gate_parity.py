@@ -108,6 +108,31 @@ def test_misaligned_views_take_the_scalar_path(dtype):
 
 
 @pytest.mark.parametrize("dtype", list(DTYPES))
+def test_per_head_vectors_off_a_16_byte_boundary(dtype):
+    """H a multiple of 8 with dt_bias and decay_scale one float into their
+    buffers: the vector path then reads them element by element."""
+    from gated_delta_rule_recurrent_b200 import last_launch, linear_attention_gate
+
+    x = workloads.make_gate_inputs((300, 4, 64), dtype, seed=78)
+    H = x["a"].shape[-1]
+    dtb = torch.zeros(H + 1, dtype=torch.float32, device="cuda")
+    dsc = torch.zeros(H + 1, dtype=torch.float32, device="cuda")
+    dtb[1:] = x["dt_bias"].cuda()
+    dsc[1:] = x["decay_scale"].cuda()
+    assert dtb[1:].data_ptr() % 16 != 0
+    decay, beta = linear_attention_gate(x["a"].cuda(), dtb[1:], dsc[1:], b=x["b"].cuda(),
+                                        want_beta=True)
+    torch.cuda.synchronize()
+    assert last_launch()["kernel"] == "gate"
+    ref_decay, ref_beta = O.linear_attention_gate(x["a"].double().numpy(),
+                                                  x["dt_bias"].double().numpy(),
+                                                  x["decay_scale"].double().numpy(),
+                                                  x["b"].double().numpy())
+    check(decay, ref_decay, dtype)
+    check(beta, ref_beta, dtype)
+
+
+@pytest.mark.parametrize("dtype", list(DTYPES))
 def test_special_values(dtype):
     """Saturation, infinities and NaN: softplus(-inf) = 0 (decay = -0.0 for a
     negative scale), softplus(+inf) = inf, sigmoid(+-inf) = 1, 0; NaN propagates."""
