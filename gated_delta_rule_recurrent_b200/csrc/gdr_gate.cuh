@@ -25,12 +25,19 @@ enum GateType { kGateF32 = 0, kGateF16 = 1, kGateBF16 = 2 };
 // library forms of gdr_decode.cuh. For a 16-bit output (one unit in the last
 // place is 2^-8 of the value for bf16, 2^-11 for fp16) cheaper forms suffice:
 //   exp and the division: the fast hardware forms (a few fp32 ulps);
-//   log1p(z), 0 <= z <= 1: z (1 - z/2) below 2^-8, where the dropped terms of
-//     the Taylor series are under z^2/3 < 2^-17 relative; log(1 + z) above,
-//     where rounding 1 + z costs at most 2^-24 / z <= 2^-16 relative and the
-//     fast logarithm's absolute error (~2^-21) at most 2^-13 relative.
+//   log1p(z), 0 <= z <= 1: z q(z), with q a degree-5 polynomial fitted to
+//     log1p(z) / z on [0, 1] by least squares at 4000 Chebyshev nodes,
+//     weighted for relative error. Evaluated by Horner's rule in fp32 its
+//     relative error is below 1e-5 (about 2^-16.6) over the whole interval,
+//     small z included, and it takes no special-function instruction.
 __device__ __forceinline__ float log1p_narrow(float z) {
-  return z < 0.00390625f ? z * fmaf(-0.5f, z, 1.0f) : __logf(1.0f + z);
+  float q = -0.02333560399711132f;
+  q = fmaf(q, z, 0.09986384958028793f);
+  q = fmaf(q, z, -0.20883141458034515f);
+  q = fmaf(q, z, 0.32475757598876953f);
+  q = fmaf(q, z, -0.4993025064468384f);
+  q = fmaf(q, z, 0.9999903440475464f);
+  return z * q;
 }
 template <bool FAST>
 __device__ __forceinline__ float gate_softplus(float x) {
