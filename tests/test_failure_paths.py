@@ -99,12 +99,14 @@ FAMILIES = [
     ("single_token", 64, 512, 4, 40, 1),
     ("chunked", 64, 512, 4, 6, 3),
     ("tensor_core", 128, 128, 4, 40, 3),
+    ("tensor_core", 128, 128, 4, 40, 8),  # the instance built for T = 8
     ("tensor_core_one", 128, 128, 4, 40, 1),
     ("prefill", 128, 128, 4, 40, 20),
 ]
 
 
-@pytest.mark.parametrize("what,D_k,D_v,H,B,T", FAMILIES, ids=[f[0] for f in FAMILIES])
+@pytest.mark.parametrize("what,D_k,D_v,H,B,T", FAMILIES,
+                         ids=[f"{f[0]}-T{f[5]}" for f in FAMILIES])
 def test_held_tile_times_out_cleanly(hooks, what, D_k, D_v, H, B, T):
     L = hooks
     pf = what == "prefill"
