@@ -90,8 +90,8 @@ def decode_kernel_name(w, layout):
     """The kernel the library launches for this workload (one per call)."""
     if w.D_k == 128 and w.D_v % 128 == 0:
         return "gdr::decode_chunk_tc_kernel"
-    if w.T == 1 and layout == "kv":
-        return "gdr::decode_tma_kernel"
+    if w.T == 1:
+        return "gdr::decode_tma_kernel" if layout == "kv" else "gdr::decode_rows_kernel"
     return "gdr::decode_chunk_kernel"
 
 

@@ -55,7 +55,7 @@ class LaunchInfo(ctypes.Structure):
 
 # gdr_kernel values of include/gdr.h
 KERNEL_NAMES = {0: "none", 1: "single_token", 2: "chunked", 3: "tensor_core",
-                4: "tensor_core_one", 5: "gate", 6: "prefill"}
+                4: "tensor_core_one", 5: "gate", 6: "prefill", 7: "rows"}
 
 _P = ctypes.c_void_p
 _DECODE_ARGTYPES = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,

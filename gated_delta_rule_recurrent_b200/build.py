@@ -29,6 +29,7 @@ TEST_HOOKS_FLAGS = ["-DGDR_TEST_HOOKS"]
 SOURCES = [os.path.join(CSRC, "gdr_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, name) for name in (
     "gdr_decode.cuh", "gdr_ptx.cuh", "gdr_decode_tma.cuh", "gdr_decode_chunk.cuh", "gdr_decode_chunk_tc.cuh",
+    "gdr_decode_rows.cuh",
     "gdr_umma.cuh", "gdr_gate.cuh", "gdr_prefill_tc.cuh")] + [
     os.path.join(INCLUDE, "gdr.h")]
 

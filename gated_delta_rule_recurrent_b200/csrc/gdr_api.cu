@@ -20,6 +20,7 @@
 #include "gdr_decode.cuh"
 #include "gdr_decode_chunk.cuh"
 #include "gdr_decode_chunk_tc.cuh"
+#include "gdr_decode_rows.cuh"
 #include "gdr_decode_tma.cuh"
 #include "gdr_gate.cuh"
 #include "gdr_prefill_tc.cuh"
@@ -401,6 +402,41 @@ int launch_chunk_tc(const gdr::DecodeParams& p, cudaStream_t stream) {
                     : launch_chunk_tc_sums<GATED, VK, false, false>(p, stream);
 }
 
+// ---------------------------------------------------------------- k-contiguous single token
+
+// One warp per block of RB rows of a head, 8 warps per CTA, as many CTAs as
+// stay resident (a grid-stride loop takes the rest). Single-token calls only.
+template <int DK, bool GATED, int RB>
+int launch_rows(const gdr::DecodeParams& p, cudaStream_t stream) {
+  if (p.T != 1 || p.D_v % RB != 0) return GDR_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(GDR_ERR_CUDA, "cudaGetDevice failed");
+  DeviceProps props;
+  int rc = device_props(dev, &props);
+  if (rc != GDR_OK) return rc;
+  static const int resident = [] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gdr::decode_rows_kernel<DK, GATED, RB>,
+                                                      gdr::kRowsThreads, 0) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    return n;
+  }();
+  const long long n_blocks = static_cast<long long>(p.B) * p.H_v * (p.D_v / RB);
+  if (n_blocks > 0x7fffffffLL) return fail(GDR_ERR_DIMS, "too many row blocks");
+  const long long warps_per_cta = gdr::kRowsThreads / 32;
+  const long long need = (n_blocks + warps_per_cta - 1) / warps_per_cta;
+  const long long cap = static_cast<long long>(props.sms) * resident;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  gdr::decode_rows_kernel<DK, GATED, RB><<<grid, gdr::kRowsThreads, 0, stream>>>(
+      p, static_cast<int>(n_blocks));
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess)
+    return fail(GDR_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(err));
+  record_launch(GDR_KERNEL_ROWS, DK, RB, GATED, true, grid, gdr::kRowsThreads, 0, 0);
+  return GDR_OK;
+}
+
 using LaunchFn = int (*)(const gdr::DecodeParams&, cudaStream_t);
 struct SliceKernel {
   int vs;
@@ -428,12 +464,18 @@ const SliceKernel* slice_kernels(int D_k, bool one, bool vk, int* n) {
   static const SliceKernel k64_many[] = {{128, launch_chunk<64, 128, GATED, false>},
                                          {64, launch_chunk<64, 64, GATED, false>}};
   static const SliceKernel k128_many[] = {{64, launch_chunk<128, 64, GATED, false>}};
-  // k-contiguous pools: the chunked kernel for every T (one token is L = 1)
+  // k-contiguous pools: one token per call takes the row kernel (blocks of 64
+  // rows, or 16 when a batch gives too few blocks), several the chunked kernel
+  static const SliceKernel k64_vk_one[] = {{64, launch_rows<64, GATED, 64>},
+                                           {16, launch_rows<64, GATED, 16>}};
+  static const SliceKernel k128_vk_one[] = {{64, launch_rows<128, GATED, 64>},
+                                            {16, launch_rows<128, GATED, 16>}};
   static const SliceKernel k64_vk[] = {{128, launch_chunk<64, 128, GATED, true>},
                                        {64, launch_chunk<64, 64, GATED, true>}};
   static const SliceKernel k128_vk[] = {{64, launch_chunk<128, 64, GATED, true>}};
   if (vk) {
-    *n = D_k == 64 ? 2 : 1;
+    *n = one ? 2 : (D_k == 64 ? 2 : 1);
+    if (one) return D_k == 64 ? k64_vk_one : k128_vk_one;
     return D_k == 64 ? k64_vk : k128_vk;
   }
   if (D_k == 64) {
@@ -500,14 +542,13 @@ std::vector<gdr_launch_info> kernel_forms() {
     for (int D_k : {64, 128})
       for (int vk = 0; vk < 2; ++vk)
         for (int one = 1; one >= 0; --one) {
-          if (vk && one) continue;  // k-contiguous pools: one table for every T
           int n = 0;
           const SliceKernel* ks = gated ? slice_kernels<true>(D_k, one, vk, &n)
                                         : slice_kernels<false>(D_k, one, vk, &n);
+          const int kernel =
+              one ? (vk ? GDR_KERNEL_ROWS : GDR_KERNEL_SINGLE_TOKEN) : GDR_KERNEL_CHUNKED;
           for (int i = 0; i < n; ++i)
-            forms.push_back(gdr_launch_info{
-                one && !vk ? GDR_KERNEL_SINGLE_TOKEN : GDR_KERNEL_CHUNKED, D_k, ks[i].vs, gated,
-                vk, 0, 0, 0, 0});
+            forms.push_back(gdr_launch_info{kernel, D_k, ks[i].vs, gated, vk, 0, 0, 0, 0});
         }
   }
   return forms;
@@ -855,7 +896,7 @@ GDR_API int gdr_kernel_form(int i, gdr_launch_info* info) {
   return GDR_OK;
 }
 
-GDR_API int gdr_abi_version(void) { return 5; }
+GDR_API int gdr_abi_version(void) { return 6; }
 
 #ifdef GDR_TEST_HOOKS
 // Test builds only (libgdr_testhooks.so): shorten the budget of the

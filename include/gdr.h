@@ -277,7 +277,8 @@ typedef enum gdr_kernel {
   GDR_KERNEL_TENSOR_CORE = 3,      /* D_k = 128, D_v a multiple of 128, several tokens */
   GDR_KERNEL_TENSOR_CORE_ONE = 4,  /* the same kernel's form for one token per call */
   GDR_KERNEL_GATE = 5,             /* the standalone gate */
-  GDR_KERNEL_PREFILL = 6           /* gdr_prefill / gdr_prefill_gated */
+  GDR_KERNEL_PREFILL = 6,          /* gdr_prefill / gdr_prefill_gated */
+  GDR_KERNEL_ROWS = 7              /* one token on a k-contiguous pool, one row per lane group */
 } gdr_kernel;
 
 /* One kernel launch: its family, the key width, the column width of a tile
@@ -309,9 +310,9 @@ GDR_API int gdr_last_launch(gdr_launch_info* info);
 GDR_API int gdr_kernel_form_count(void);
 GDR_API int gdr_kernel_form(int i, gdr_launch_info* info);
 
-/* Library ABI version, currently 5 (2 added gdr_linear_attention_gate, 3 the
+/* Library ABI version, currently 6 (2 added gdr_linear_attention_gate, 3 the
  * layout field of gdr_dims, 4 gdr_last_launch and the kernel forms, 5
- * gdr_prefill and gdr_prefill_gated). */
+ * gdr_prefill and gdr_prefill_gated, 6 the GDR_KERNEL_ROWS form). */
 GDR_API int gdr_abi_version(void);
 
 #ifdef __cplusplus

@@ -45,6 +45,10 @@ CASES = [
     ("tensor_core_one", 128, 128, "vk", 1, 256, 4),
     ("tensor_core", 128, 128, "vk", 5, 256, 4),
     ("tensor_core", 128, 128, "vk", 8, 256, 4),
+    ("rows", 64, 64, "vk", 1, 512, 64),
+    ("rows", 64, 16, "vk", 1, 512, 64),
+    ("rows", 128, 64, "vk", 1, 192, 64),
+    ("rows", 128, 16, "vk", 1, 192, 4),
     ("single_token", 64, 512, "kv", 1, 512, 64),
     ("single_token", 64, 256, "kv", 1, 512, 64),
     ("single_token", 64, 128, "kv", 1, 512, 64),
@@ -52,7 +56,7 @@ CASES = [
     ("chunked", 64, 128, "kv", 4, 512, 64),
     ("chunked", 64, 64, "kv", 4, 512, 64),
     ("chunked", 64, 128, "vk", 3, 512, 64),
-    ("chunked", 64, 64, "vk", 1, 512, 64),
+    ("chunked", 64, 64, "vk", 2, 512, 64),
     ("single_token", 128, 64, "kv", 1, 192, 4),
     ("chunked", 128, 64, "kv", 6, 192, 4),
     ("chunked", 128, 64, "vk", 2, 192, 4),
@@ -60,7 +64,8 @@ CASES = [
 
 # tile widths of the width-chosen tables, widest first
 WIDTHS = {("single_token", 64, "kv"): (512, 256, 128, 64), ("chunked", 64, "kv"): (128, 64),
-          ("chunked", 64, "vk"): (128, 64)}
+          ("chunked", 64, "vk"): (128, 64), ("rows", 64, "vk"): (64, 16),
+          ("rows", 128, "vk"): (64, 16)}
 
 
 def case_key(case, gated):

@@ -49,7 +49,7 @@ def test_status_strings_and_version(built_library):
     from gated_delta_rule_recurrent_b200 import binding
 
     L = binding.lib()
-    assert L.gdr_abi_version() == 5
+    assert L.gdr_abi_version() == 6
     for code, name in binding.STATUS_NAMES.items():
         assert L.gdr_status_string(code).decode() == name
     assert L.gdr_status_string(99).decode() == "unknown status"
