@@ -273,7 +273,7 @@ GDR_API int gdr_device_error(uint32_t* flags, int reset);
 typedef enum gdr_kernel {
   GDR_KERNEL_NONE = 0,
   GDR_KERNEL_SINGLE_TOKEN = 1,     /* one token per call, CUDA cores */
-  GDR_KERNEL_CHUNKED = 2,          /* several tokens (or a k-contiguous pool), CUDA cores */
+  GDR_KERNEL_CHUNKED = 2,          /* several tokens, CUDA cores */
   GDR_KERNEL_TENSOR_CORE = 3,      /* D_k = 128, D_v a multiple of 128, several tokens */
   GDR_KERNEL_TENSOR_CORE_ONE = 4,  /* the same kernel's form for one token per call */
   GDR_KERNEL_GATE = 5,             /* the standalone gate */
@@ -282,8 +282,9 @@ typedef enum gdr_kernel {
 } gdr_kernel;
 
 /* One kernel launch: its family, the key width, the column width of a tile
- * (0 for the gate), whether the gate is fused, the pool layout, and the launch
- * shape (blocks, threads per block, dynamic shared memory, pipeline stages). */
+ * (the rows of a warp's block for GDR_KERNEL_ROWS; 0 for the gate), whether
+ * the gate is fused, the pool layout, and the launch shape (blocks, threads
+ * per block, dynamic shared memory, pipeline stages). */
 typedef struct gdr_launch_info {
   int32_t kernel;
   int32_t D_k;
