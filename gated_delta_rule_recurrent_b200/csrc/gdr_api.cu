@@ -448,8 +448,10 @@ struct SliceKernel {
 // thread count of a block caps the registers ptxas may give a thread (255 up
 // to 256 threads, 168 up to 384, 128 up to 512, 96 up to 640), and a
 // single-token call keeps no state in registers (about 75 of them), so a
-// full-width 64 x 512 tile can use 16 consumer warps. Multi-token calls use
-// the CUDA-core chunked kernel. These tables serve the calls the tensor-core
+// full-width 64 x 512 tile can use 16 consumer warps. Single-token calls on
+// a k-contiguous pool use the row kernel, whose "width" is the rows of a
+// warp's block (64, or 16 for small batches). Multi-token calls use the
+// CUDA-core chunked kernel. These tables serve the calls the tensor-core
 // kernel does not take (D_k = 64, or D_v not a multiple of 128), and are its
 // fallback.
 template <bool GATED>
